@@ -1,0 +1,485 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged decode-attention step on B200.
+
+One step = the whole hot path over one decode batch: write each sequence's
+new token into its cache slot (pa_reshape_and_cache; pa_copy_blocks when a
+step needs a copy-on-write), then decode attention through the block tables
+(pa_decode). Default workload: 64 sequences, 32/32 heads, head_dim 128,
+bf16 KV, context lengths U[512, 2048] (the Llama-7B-shaped layer).
+
+Prints ONE JSON line (rank 0). `value` is the achieved HBM GB/s of the step
+(algorithmic bytes: K/V of every context token, q, out, table entries and
+the new-token write, over the device time), summed over ranks; `e2e` is the
+same metric with the step's inputs copied from pinned host memory and the
+output copied back, every step; `roofline` is the decode kernel alone.
+
+  python bench.py [--gpus N --steps K --warmup W --workload NAME --impl ours|reference]
+
+With torchrun (N > 1) every rank decodes its own batch (its own sequences,
+its own pool; no collective on the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of B200 peak), decode tokens/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+DECODE_SOURCES = ["paged_kv_cache_429_b200/csrc/decode.cuh",
+                  "paged_kv_cache_429_b200/csrc/ptx.cuh"]
+
+
+# ----------------------------------------------------------------- helpers
+
+def describe(w: synth.Workload) -> str:
+    if w.prefix_len:
+        lens = f"shared {w.prefix_len}-token prefix + lognormal(median {w.suffix_median:g}) suffix"
+    else:
+        lens = f"L~U[{w.len_lo},{w.len_hi}]"
+    kv = "fp8_e4m3" if w.kv_fp8 else "bf16"
+    return (f"{w.name}: {w.num_seqs} seqs, {w.num_q_heads}/{w.num_kv_heads} heads, "
+            f"d{w.head_dim}, {kv} KV, block 16, {lens}")
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            peaks = json.load(f)
+        return float(peaks["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary of this
+    workload, if it was taken on the current decode kernel source."""
+    path = os.path.join(ROOT, "profiles", f"paged_decode_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (m_hash and m_tr) or m_hash.group(1) != decode_source_hash():
+        return None
+    return int(m_tr.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting",
+               0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x10: "sync_boost",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks
+            self.nv, self.error = None, repr(e)
+
+    def _handle(self, idx):
+        nv = self.nv
+        try:
+            props = torch.cuda.get_device_properties(idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId_v2(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _sample(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(mhz)
+        for b, name in self.REASONS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world, device):
+    if world > 1:
+        import torch.distributed as dist
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_timing(elapsed_ms: float, nbytes: float, world: int, device):
+    """(max elapsed ms over ranks, total bytes over ranks)."""
+    if world == 1:
+        return elapsed_ms, nbytes
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
+    b = torch.tensor([nbytes], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b.item())
+
+
+# ------------------------------------------------------------- our GPU arm
+
+def run_ours(args, world, rank, local):
+    from paged_kv_cache_429_b200.batch import DecodeBatch
+
+    device = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload]
+    if args.partition_size is not None:
+        import dataclasses
+        w = dataclasses.replace(w, partition_size=args.partition_size)
+    batch = DecodeBatch.build(w, args.seed + rank, device)
+    stream = torch.cuda.current_stream(device)
+    ps = w.partition_size
+    ws = batch.workspace(ps if ps != 0 else 0)
+
+    step_writes = sum((op.row1 - op.row0) for op in batch.step_ops if op.kind == "write")
+    eb = 1 if w.kv_fp8 else 2
+    reshape_bytes = step_writes * w.num_kv_heads * w.head_dim * (2 * 2 + 2 * eb) + 8 * step_writes
+    decode_bytes = batch.algorithmic_bytes()
+    step_bytes = decode_bytes + reshape_bytes
+    n_copy_launches = sum(1 for op in batch.step_ops if op.kind == "copy")
+    n_write_launches = sum(1 for op in batch.step_ops if op.kind == "write")
+
+    def one_step(ev=None):
+        batch.run_ops(batch.step_ops)
+        if ev is not None:
+            ev[0].record(stream)
+        batch.decode(partition_size=ps, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # which decode path runs (split launches a second, reduce kernel)
+    split = ps > 0 or (ps < 0 and ws is not None and _auto_split(batch, ws))
+    launches_per_step = n_write_launches + n_copy_launches + (2 if split else 1)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(device)
+
+    # ---- device-resident timing
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        one_step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    barrier(world, device)
+    elapsed = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    max_ms, total_bytes = reduce_timing(elapsed, step_bytes * K, world, device)
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    ms_per_step = max_ms / K
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+
+    # ---- end to end: pinned host inputs in, output back, every step
+    e2e = run_e2e(batch, args, ps, ws, stream, device, world, step_bytes)
+
+    if rank != 0:
+        return None
+    peak, peak_src = measured_peak()
+    achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if w.kv_fp8 else "bf16", "data": "synthetic",
+        "config": {
+            "workload": describe(w), "global_batch": w.num_seqs * world,
+            "seq_len": f"U[{w.len_lo},{w.len_hi}]" if not w.prefix_len else "prefix+suffix",
+            "parallelism": f"dp{world} (independent sequence shards, no collective)",
+            "decode_path": "split-context" if split else "single-pass",
+            "partition_size": ps,
+            "l2": (f"inputs larger than L2: {decode_bytes / 1e9:.2f} GB per step vs "
+                   f"{L2_BYTES / 2**20:.0f} MiB L2; no flush"),
+            "seed": args.seed,
+        },
+        "tokens_per_s": round(w.num_seqs * world / (ms_per_step * 1e-3), 1),
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "pct_of_8tbs_datasheet": round(100 * value / world / 8000.0, 2),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(w.name),
+                     "kernel": "paged_decode_kernel" + (" + reduce" if split else ""),
+                     "algorithmic_bytes_per_launch": decode_bytes,
+                     "avg_launch_ms": round(dec_avg_ms, 6), "peak_source": peak_src},
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(batch, args.cpu_seconds)
+    return line
+
+
+def _auto_split(batch, ws) -> bool:
+    """Mirror of the library's automatic choice, for reporting only."""
+    w = batch.w
+    sms = torch.cuda.get_device_properties(batch.device).multi_processor_count
+    units = w.num_seqs * w.num_kv_heads
+    cap = min(batch.max_context_len, batch.max_blocks * 16)
+    return (units < 6 * sms or cap > 4096) and cap > 512
+
+
+def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):
+    """Same step through the public API with host buffers: every step copies
+    q, the new K/V, slots, block tables and context lengths from pinned host
+    memory, runs the step, and reads the output back."""
+    b = batch
+    new_op = [op for op in b.step_ops if op.kind == "write"][0]
+    slot_dev = b._dev_slots[id(new_op)]
+    host = {
+        "q": b.q.cpu().pin_memory(), "k_new": b.k_new.cpu().pin_memory(),
+        "v_new": b.v_new.cpu().pin_memory(), "slots": slot_dev.cpu().pin_memory(),
+        "tables": b.block_tables.cpu().pin_memory(),
+        "lens": b.context_lens.cpu().pin_memory(),
+    }
+    dev = {"q": b.q, "k_new": b.k_new, "v_new": b.v_new, "slots": slot_dev,
+           "tables": b.block_tables, "lens": b.context_lens}
+    out_host = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            dev[k].copy_(t, non_blocking=True)
+        b.step(partition_size=ps, workspace=ws)
+        out_host.copy_(b.out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    K = max(1, args.steps // 4)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    t0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    max_ms, total = reduce_timing(t0.elapsed_time(t1), step_bytes * K, world, device)
+    return {"value": round(total / (max_ms * 1e-3) / 1e9, 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": round(max_ms / K, 6)}
+
+
+# ------------------------------------------------------- CPU oracle timing
+
+def oracle_host_inputs(w: synth.Workload, seed: int):
+    """Host-only inputs of the workload's shape for the oracle: lengths from
+    synth, each sequence's blocks taken in order from a seeded permutation
+    of the pool, every pool slot filled with N(0,1) bf16 values."""
+    lens = synth.draw_lengths(w, seed)
+    nblk = -(-lens // 16)
+    nb = w.pool_blocks or int(np.ceil(w.pool_factor * nblk.sum()))
+    perm = synth.rng(seed, w.name, "pool").permutation(nb).astype(np.int32)
+    tables = np.full((w.num_seqs, int(nblk.max())), -1, np.int32)
+    k = 0
+    for s in range(w.num_seqs):
+        tables[s, :nblk[s]] = perm[k:k + nblk[s]]
+        k += nblk[s]
+    shape = (nb, w.num_kv_heads, 16, w.head_dim)
+    kc = synth.randn_bf16(shape, seed, w.name, "k_old").view(torch.int16).numpy().view(np.uint16)
+    vc = synth.randn_bf16(shape, seed, w.name, "v_old").view(torch.int16).numpy().view(np.uint16)
+    q = synth.randn_bf16((w.num_seqs, w.num_q_heads, w.head_dim), seed, w.name,
+                         "q").view(torch.int16).numpy().view(np.uint16)
+    return lens, tables, kc, vc, q
+
+
+def seq_bytes(w, L):
+    eb = 1 if w.kv_fp8 else 2
+    return (L * w.num_kv_heads * w.head_dim * eb * 2 + w.num_q_heads * w.head_dim * 6
+            + (-(-L // 16)) * 4 + 4)
+
+
+def time_oracle(w, inputs, budget_s: float, steps=None):
+    """Oracle decode, one sequence per step (round robin), on this host's
+    cores (the oracle is single-threaded). Returns (GB/s, steps, seconds)."""
+    import oracle
+    lens, tables, kc, vc, q = inputs
+    n, nbytes, t_total = 0, 0, 0.0
+    while True:
+        s = n % w.num_seqs
+        t = time.perf_counter()
+        oracle.paged_decode(q, kc, vc, tables, lens.astype(np.int32), w.sm_scale,
+                            seq_subset=[s])
+        t_total += time.perf_counter() - t
+        nbytes += seq_bytes(w, int(lens[s]))
+        n += 1
+        if (steps is not None and n >= steps) or (steps is None and t_total >= budget_s):
+            break
+    return nbytes / t_total / 1e9, n, t_total
+
+
+def cpu_baseline(batch, budget_s):
+    w = batch.w
+    inputs = oracle_host_inputs(w, batch.seed)
+    gbs, n, secs = time_oracle(w, inputs, budget_s)
+    return {"value": round(gbs, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": (f"{n} single-sequence decode steps of the {w.name} workload "
+                       f"(round robin over its {w.num_seqs} sequences), {secs:.1f} s "
+                       f"of single-threaded fp64 oracle time; host has "
+                       f"{os.cpu_count()} cores")}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    inputs = oracle_host_inputs(w, args.seed)
+    time_oracle(w, inputs, 0, steps=max(1, args.warmup))
+    gbs, n, secs = time_oracle(w, inputs, 0, steps=max(1, args.steps))
+    ms_per_step = secs / n * 1e3
+    sample = (f"one sequence per step (round robin over the {w.num_seqs} sequences of "
+              f"the {w.name} workload), single-threaded fp64 oracle; host has "
+              f"{os.cpu_count()} cores")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 6), "unit": UNIT,
+        "n_gpus": world, "steps": n, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(w), "global_batch": w.num_seqs,
+                   "parallelism": "single host thread"},
+        "cpu_baseline": {"value": round(gbs, 6), "unit": UNIT, "cores": 1,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        # the CPU oracle arm: rank 0 alone runs it, other ranks exit at once
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = init_dist()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    try:
+        line = run_ours(args, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,112 @@
+// Cache writes for the paged KV cache.
+//
+// reshape_and_cache — "第 7 章推理框架：vLLM 与 PagedAttention" §7.1
+// ("Block 与 Block Table": a generated token's K/V goes into the next slot,
+// a new block after 16) and "GPU 学习日报 Day 28" §4.2 / FAQ Q4 (prefill
+// KV is written block-wise into the pool too). Each thread moves one
+// 16-byte chunk (8 elements) of one (token, KV head) row; a warp covers
+// whole rows, so reads and writes are coalesced 16-byte accesses.
+//
+// copy_blocks — copy-on-write of a shared block ("vLLM 与 PagedAttention：
+// 把 GPU 显存当操作系统内存管" §PagedAttention 写时复制; Day 28 §六 item 4).
+// Each CTA streams one (pair, cache) block with 16-byte loads/stores.
+#pragma once
+
+#include <cuda_fp8.h>
+#include <cstdint>
+
+#include "decode.cuh"
+
+namespace pa {
+
+constexpr int kCacheThreads = 256;
+
+template <bool FP8>
+__global__ void __launch_bounds__(kCacheThreads)
+    reshape_and_cache_kernel(const uint4 *__restrict__ key,
+                             const uint4 *__restrict__ value, void *k_cache,
+                             void *v_cache, const int64_t *__restrict__ slots,
+                             int64_t total_chunks, int chunks_per_token,
+                             int chunks_per_row, int num_kv_heads, int head_dim,
+                             int64_t num_slots, float k_scale, float v_scale) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+       i < total_chunks; i += stride) {
+    const int64_t t = i / chunks_per_token;
+    const int rem = static_cast<int>(i - t * chunks_per_token);
+    const int h = rem / chunks_per_row;
+    const int c = rem - h * chunks_per_row;
+    const int64_t slot = slots[t];
+    if (slot < 0) continue;
+    if (slot >= num_slots) {
+      if (c == 0 && h == 0) raise_error(kErrSlotRange);
+      continue;
+    }
+    const int64_t blk = slot / kBS;
+    const int off = static_cast<int>(slot - blk * kBS);
+    // element index of the chunk inside the cache
+    const int64_t dst = ((blk * num_kv_heads + h) * kBS + off) * head_dim + c * 8;
+    const uint4 kx = key[i];
+    const uint4 vx = value[i];
+    if constexpr (!FP8) {
+      *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(k_cache) + dst) = kx;
+      *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(v_cache) + dst) = vx;
+    } else {
+      const uint32_t kw[4] = {kx.x, kx.y, kx.z, kx.w};
+      const uint32_t vw[4] = {vx.x, vx.y, vx.z, vx.w};
+      uint32_t ko[2], vo[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t kb = 0, vb = 0;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t kwe = kw[2 * j + e], vwe = vw[2 * j + e];
+          // y = x / scale, IEEE binary32 division, then E4M3 RNE + satfinite
+          const float2 ky = make_float2(__fdiv_rn(__uint_as_float(kwe << 16), k_scale),
+                                        __fdiv_rn(__uint_as_float(kwe & 0xFFFF0000u), k_scale));
+          const float2 vy = make_float2(__fdiv_rn(__uint_as_float(vwe << 16), v_scale),
+                                        __fdiv_rn(__uint_as_float(vwe & 0xFFFF0000u), v_scale));
+          const uint32_t kq = __nv_cvt_float2_to_fp8x2(ky, __NV_SATFINITE, __NV_E4M3);
+          const uint32_t vq = __nv_cvt_float2_to_fp8x2(vy, __NV_SATFINITE, __NV_E4M3);
+          kb |= (kq & 0xFFFFu) << (16 * e);
+          vb |= (vq & 0xFFFFu) << (16 * e);
+        }
+        ko[j] = kb;
+        vo[j] = vb;
+      }
+      *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(k_cache) + dst) = make_uint2(ko[0], ko[1]);
+      *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(v_cache) + dst) = make_uint2(vo[0], vo[1]);
+    }
+  }
+}
+
+// grid.x = 2 * num_pairs (pair i: CTA 2i copies K, 2i+1 copies V)
+__global__ void __launch_bounds__(kCacheThreads)
+    copy_blocks_kernel(uint4 *k_cache, uint4 *v_cache,
+                       const int64_t *__restrict__ pairs, int64_t block_chunks,
+                       int num_blocks) {
+  const int pair = blockIdx.x >> 1;
+  uint4 *cache = (blockIdx.x & 1) ? v_cache : k_cache;
+  const int64_t src = pairs[2 * pair];
+  const int64_t dst = pairs[2 * pair + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && (blockIdx.x & 1) == 0) raise_error(kErrPairRange);
+    return;
+  }
+  const uint4 *s = cache + src * block_chunks;
+  uint4 *d = cache + dst * block_chunks;
+  int64_t i = threadIdx.x;
+  for (; i + 3 * kCacheThreads < block_chunks; i += 4 * kCacheThreads) {
+    const uint4 x0 = s[i];
+    const uint4 x1 = s[i + kCacheThreads];
+    const uint4 x2 = s[i + 2 * kCacheThreads];
+    const uint4 x3 = s[i + 3 * kCacheThreads];
+    d[i] = x0;
+    d[i + kCacheThreads] = x1;
+    d[i + 2 * kCacheThreads] = x2;
+    d[i + 3 * kCacheThreads] = x3;
+  }
+  for (; i < block_chunks; i += kCacheThreads) d[i] = s[i];
+}
+
+}  // namespace pa

@@ -1,0 +1,355 @@
+// C ABI of libpa.so: argument checks, TMA descriptor set-up and launches.
+// Declarations and the contract of every entry point: include/pa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa.h"
+#include "cache_ops.cuh"
+#include "decode.cuh"
+
+namespace {
+
+using pa::DecodeParams;
+using pa::Geo;
+using pa::ReduceParams;
+
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultPartition = 512;
+
+bool aligned(const void *ptr, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
+}
+
+// --- driver entry point for tensor-map encoding (no link against libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+int device_sm_count(int dev) {
+  static std::atomic<int> cache[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+// Tensor map over one cache viewed as a 2-D array [num_blocks*Hkv*16][D].
+template <int D, bool FP8>
+bool make_cache_tmap(CUtensorMap *map, const void *base, int rows) {
+  using G = Geo<D, FP8>;
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(G::kRowBytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(G::kBoxRow / G::kEB), static_cast<cuuint32_t>(pa::kBS)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      G::kBoxRow == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = enc(map, FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8, int NT>
+size_t decode_smem_bytes() {
+  using G = Geo<D, FP8>;
+  return 1024 + G::kRingBytes + 16 * G::kStages + 16;
+}
+
+template <typename Kern>
+bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int dev) {
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_relaxed) & bit) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess)
+    return false;
+  done.fetch_or(bit, std::memory_order_relaxed);
+  return true;
+}
+
+template <int D, bool FP8, int NT>
+pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
+                        const DecodeParams &p, int num_seqs, int grid_x,
+                        cudaStream_t stream, int dev) {
+  CUtensorMap tk, tv;
+  if (!make_cache_tmap<D, FP8>(&tk, k_cache, rows) ||
+      !make_cache_tmap<D, FP8>(&tv, v_cache, rows))
+    return PA_ERR_CUDA;
+  auto kern = pa::paged_decode_kernel<D, FP8, NT>;
+  static std::atomic<uint64_t> attr_done{0};
+  const size_t smem = decode_smem_bytes<D, FP8, NT>();
+  if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
+  dim3 grid(grid_x, p.num_kv_heads, num_seqs);
+  kern<<<grid, pa::kDecodeThreads, smem, stream>>>(tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D>
+pa_status launch_reduce(const ReduceParams &r, int num_seqs, cudaStream_t stream, int dev) {
+  auto kern = pa::paged_decode_reduce_kernel<D>;
+  const size_t smem = static_cast<size_t>(r.max_partitions) * sizeof(float);
+  static std::atomic<uint64_t> attr_done{0};
+  if (smem > 48 * 1024) {
+    if (!ensure_smem_attr(kern, 227 * 1024, attr_done, dev)) return PA_ERR_CUDA;
+  }
+  dim3 grid(r.num_q_heads, num_seqs);
+  kern<<<grid, D, smem, stream>>>(r);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, bool FP8>
+pa_status dispatch_nt(int nt, const void *kc, const void *vc, int rows, const DecodeParams &p,
+                      int num_seqs, int grid_x, cudaStream_t st, int dev) {
+  return nt == 1 ? launch_decode<D, FP8, 1>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                 : launch_decode<D, FP8, 2>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+}
+
+size_t workspace_bytes_for(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                           int psize) {
+  const int64_t P = (static_cast<int64_t>(max_context_len) + psize - 1) / psize;
+  const int64_t floats = static_cast<int64_t>(num_seqs) * num_q_heads * P * (head_dim + 2);
+  const int64_t bytes = floats * 4 + 2 * 256;  // two sub-array alignments
+  return static_cast<size_t>((bytes + 255) / 256 * 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_OUT_OF_BLOCKS: return "PA_ERR_OUT_OF_BLOCKS";
+    case PA_ERR_NOT_FOUND: return "PA_ERR_NOT_FOUND";
+    case PA_ERR_DEVICE: return "PA_ERR_DEVICE";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+                                int max_context_len, int partition_size) {
+  if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0)
+    return 0;
+  if (partition_size == 0) return 0;
+  const int psize = partition_size < 0 ? kDefaultPartition : partition_size;
+  if (psize % pa::kBS != 0) return 0;
+  return workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_context_len, psize);
+}
+
+pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+                    pa_kv_dtype kv_dtype, float k_scale, float v_scale,
+                    const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, int max_context_len, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float sm_scale, int partition_size, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  // ---- shape and pointer checks (host only; nothing launched on error)
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_blocks_per_seq < 0 || max_context_len < 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (!std::isfinite(sm_scale)) return PA_ERR_INVALID_ARG;
+  if (kv_dtype == PA_KV_FP8_E4M3 &&
+      !(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
+  if (partition_size < -1 || (partition_size > 0 && partition_size % pa::kBS != 0))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return PA_ERR_INVALID_ARG;
+  const int64_t rows64 = static_cast<int64_t>(num_blocks) * num_kv_heads * pa::kBS;
+  if (rows64 + pa::kBS >= INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(num_seqs) > 65535) return PA_ERR_UNSUPPORTED;  // grid.z
+  if (num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;                     // grid.y
+
+  const int ctx_cap = static_cast<int>(
+      std::min<int64_t>(max_context_len, static_cast<int64_t>(max_blocks_per_seq) * pa::kBS));
+  if (partition_size > 0) {  // forced split: the workspace must fit (host check)
+    const int64_t P = (static_cast<int64_t>(ctx_cap) + partition_size - 1) / partition_size;
+    if (P > 65535 || P * 4 > 200 * 1024) return PA_ERR_UNSUPPORTED;
+    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap,
+                                            partition_size);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+      return PA_ERR_WORKSPACE;
+  }
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // ---- path choice
+  int psize = partition_size;
+  if (psize < 0) {
+    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
+    const bool wide = units >= 6LL * device_sm_count(dev);
+    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap,
+                                            kDefaultPartition);
+    const bool have_ws = workspace && aligned(workspace, 256) && workspace_bytes >= need;
+    psize = (!wide || ctx_cap > 4096) && have_ws && ctx_cap > kDefaultPartition
+                ? kDefaultPartition
+                : 0;
+  }
+
+  DecodeParams p{};
+  p.out = out;
+  p.q = static_cast<const uint16_t *>(q);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.num_blocks = num_blocks;
+  const float log2e = 1.4426950408889634f;
+  if (kv_dtype == PA_KV_BF16) {
+    p.score_scale = sm_scale * log2e;
+    p.out_scale = 1.f;
+  } else {
+    p.score_scale = sm_scale * k_scale * log2e;
+    p.out_scale = v_scale;
+  }
+  int grid_x = 1;
+  int64_t P = 1;
+  if (psize > 0) {
+    P = (static_cast<int64_t>(ctx_cap) + psize - 1) / psize;
+    if (P == 0) P = 1;
+    if (P > 65535 || P * 4 > 200 * 1024) return PA_ERR_UNSUPPORTED;
+    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap, psize);
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
+      return PA_ERR_WORKSPACE;
+    const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads * P;
+    char *ws = static_cast<char *>(workspace);
+    const size_t o_bytes = (static_cast<size_t>(rows) * head_dim * 4 + 255) / 256 * 256;
+    const size_t m_bytes = (static_cast<size_t>(rows) * 4 + 255) / 256 * 256;
+    p.ws_o = reinterpret_cast<float *>(ws);
+    p.ws_m = reinterpret_cast<float *>(ws + o_bytes);
+    p.ws_l = reinterpret_cast<float *>(ws + o_bytes + m_bytes);
+    p.partition_blocks = psize / pa::kBS;
+    p.max_partitions = static_cast<int>(P);
+    grid_x = static_cast<int>(P);
+  }
+
+  const int nt = group <= 8 ? 1 : 2;
+  const int rows = static_cast<int>(rows64);
+  pa_status rc;
+  if (kv_dtype == PA_KV_BF16)
+    rc = head_dim == 128 ? dispatch_nt<128, false>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
+                         : dispatch_nt<64, false>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
+  else
+    rc = head_dim == 128 ? dispatch_nt<128, true>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
+                         : dispatch_nt<64, true>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
+  if (rc != PA_OK || psize == 0) return rc;
+
+  ReduceParams r{};
+  r.out = out;
+  r.ws_o = p.ws_o;
+  r.ws_m = p.ws_m;
+  r.ws_l = p.ws_l;
+  r.context_lens = context_lens;
+  r.max_context_len = max_context_len;
+  r.max_blocks_per_seq = max_blocks_per_seq;
+  r.num_q_heads = num_q_heads;
+  r.partition_tokens = psize;
+  r.max_partitions = static_cast<int>(P);
+  return head_dim == 128 ? launch_reduce<128>(r, num_seqs, st, dev)
+                         : launch_reduce<64>(r, num_seqs, st, dev);
+}
+
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                               void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               pa_kv_dtype kv_dtype, float k_scale, float v_scale,
+                               void *stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (kv_dtype == PA_KV_FP8_E4M3 &&
+      !(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return PA_ERR_INVALID_ARG;
+  const int chunks_per_row = head_dim / 8;
+  const int chunks_per_token = chunks_per_row * num_kv_heads;
+  const int64_t total = static_cast<int64_t>(num_tokens) * chunks_per_token;
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * pa::kBS;
+  int64_t blocks = (total + pa::kCacheThreads - 1) / pa::kCacheThreads;
+  if (blocks > 1 << 20) blocks = 1 << 20;  // grid-stride beyond this
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kv_dtype == PA_KV_BF16)
+    pa::reshape_and_cache_kernel<false><<<static_cast<unsigned>(blocks), pa::kCacheThreads, 0, st>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), k_cache, v_cache,
+        slot_mapping, total, chunks_per_token, chunks_per_row, num_kv_heads, head_dim, num_slots,
+        1.f, 1.f);
+  else
+    pa::reshape_and_cache_kernel<true><<<static_cast<unsigned>(blocks), pa::kCacheThreads, 0, st>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), k_cache, v_cache,
+        slot_mapping, total, chunks_per_token, chunks_per_row, num_kv_heads, head_dim, num_slots,
+        k_scale, v_scale);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pairs, int num_pairs,
+                         size_t block_bytes, int num_blocks, void *stream) {
+  if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 || block_bytes % 16 != 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_pairs) return PA_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return PA_ERR_INVALID_ARG;
+  if (num_pairs > (1 << 30)) return PA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  pa::copy_blocks_kernel<<<2 * num_pairs, pa::kCacheThreads, 0, st>>>(
+      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_pairs,
+      static_cast<int64_t>(block_bytes / 16), num_blocks);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_get_device_error(uint32_t *code_out) {
+  if (!code_out) return PA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_pa_error, sizeof v) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(pa::g_pa_error, &zero, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+  *code_out = v;
+  return v ? PA_ERR_DEVICE : PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_429_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 0x100000  # aligned non-null address; never dereferenced by these calls
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PA_API[^;(]*?\b(pa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
+                     "pa_decode_workspace_size", "pa_status_string",
+                     "pa_pool_create", "pa_pool_append", "pa_pool_fork"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_exactly_the_header():
+    assert sorted(_lib.SIGNATURES) == declared_functions()
+
+
+def test_status_strings():
+    lib = _lib.lib()
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.pa_status_string(code).decode() == name
+    assert lib.pa_status_string(99).decode() == "PA_ERR_UNKNOWN"
+
+
+def test_workspace_size_formula():
+    lib = _lib.lib()
+    # 8 seqs, 64 heads, d128, 131072 tokens, 512-token partitions
+    P = 131072 // 512
+    floats = 8 * 64 * P * (128 + 2)
+    expect = (floats * 4 + 512 + 255) // 256 * 256
+    assert lib.pa_decode_workspace_size(8, 64, 128, 131072, 512) == expect
+    assert lib.pa_decode_workspace_size(8, 64, 128, 131072, -1) == expect
+    assert lib.pa_decode_workspace_size(8, 64, 128, 131072, 0) == 0
+    assert lib.pa_decode_workspace_size(8, 64, 128, 131072, 100) == 0
+
+
+def decode_args(**kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, dtype=0, ks=1.0, vs=1.0, bt=FAKE,
+             maxb=8, cl=FAKE, maxctx=128, S=2, Hq=8, Hkv=8, D=128, B=16, NB=64,
+             scale=0.1, psize=512, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(S=0), OK),                       # empty batch: nothing to launch
+    (dict(B=8), UNSUPPORTED),
+    (dict(D=96), UNSUPPORTED),
+    (dict(Hq=12, Hkv=8), UNSUPPORTED),     # not a whole group
+    (dict(Hq=32, Hkv=1), UNSUPPORTED),     # group 32 > 16
+    (dict(out=None), INVALID),
+    (dict(q=FAKE + 2), INVALID),           # misaligned
+    (dict(dtype=1, ks=0.0), INVALID),      # fp8 needs positive scales
+    (dict(dtype=1, vs=float("inf")), INVALID),
+    (dict(dtype=5), INVALID),
+    (dict(psize=100), INVALID),            # not a multiple of 16
+    (dict(psize=-2), INVALID),
+    (dict(scale=float("nan")), INVALID),
+    (dict(NB=0), INVALID),
+    (dict(psize=512, ws=None), WORKSPACE),  # forced split, no workspace
+    (dict(psize=512, ws=FAKE, wsb=1024), WORKSPACE),
+    (dict(psize=512, ws=FAKE + 16, wsb=1 << 30), WORKSPACE),  # not 256-aligned
+])
+def test_decode_rejects_bad_arguments_on_host(kw, expect):
+    assert _lib.lib().pa_decode(*decode_args(**kw)) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(T=0), OK),
+    (dict(B=32), UNSUPPORTED),
+    (dict(D=80), UNSUPPORTED),
+    (dict(key=None), INVALID),
+    (dict(slots=None), INVALID),
+    (dict(dtype=1, ks=-1.0), INVALID),
+    (dict(k=FAKE + 8), INVALID),
+])
+def test_reshape_rejects_bad_arguments_on_host(kw, expect):
+    a = dict(key=FAKE, value=FAKE, k=FAKE, v=FAKE, slots=FAKE, T=4, Hkv=8, D=128,
+             B=16, NB=64, dtype=0, ks=1.0, vs=1.0, stream=None)
+    a.update(kw)
+    assert _lib.lib().pa_reshape_and_cache(*a.values()) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(n=0), OK),
+    (dict(pairs=None), INVALID),
+    (dict(bb=1000), INVALID),   # not a multiple of 16
+    (dict(bb=0), INVALID),
+    (dict(k=FAKE + 4), INVALID),
+])
+def test_copy_rejects_bad_arguments_on_host(kw, expect):
+    a = dict(k=FAKE, v=FAKE, pairs=FAKE, n=3, bb=4096, NB=64, stream=None)
+    a.update(kw)
+    assert _lib.lib().pa_copy_blocks(*a.values()) == expect
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libpa.so"))
+    with pytest.raises(_lib.LibraryNotBuilt):
+        _lib.lib()
