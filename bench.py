@@ -216,6 +216,9 @@ def run_ours(args, world, rank, local):
         import dataclasses
         w = dataclasses.replace(w, partition_size=args.partition_size)
     batch = DecodeBatch.build(w, args.seed + rank, device)
+    # the earlier tokens' source rows were only needed to fill the cache
+    batch.k_old = batch.v_old = None
+    torch.cuda.empty_cache()
     stream = torch.cuda.current_stream(device)
     ps = w.partition_size
     ws = batch.workspace(ps if ps != 0 else 0)
