@@ -134,6 +134,42 @@ PA_API pa_status pa_decode(float *out, const void *q, const void *k_cache,
                     int num_blocks, float sm_scale, int partition_size,
                     void *workspace, size_t workspace_bytes, void *stream);
 
+/* Split-context decode for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call; it exists for the runtime
+ * around the kernels. Some callers have no device allocator to hand: a C
+ * host program or plugin that is given its input and output buffers but no
+ * way to get scratch, or a serving loop that forbids allocation after
+ * start-up because cudaMalloc/cudaFree can synchronise the device and stall
+ * other streams. This call is pa_decode with the split-context path forced
+ * (partition_size: a positive multiple of 16) and with the workspace taken
+ * from a fixed array of PA_NO_ALLOC_SCRATCH_BYTES compiled into the library
+ * instead of from the caller; every other argument means what it means for
+ * pa_decode. The call allocates nothing.
+ *   - The array occupies PA_NO_ALLOC_SCRATCH_BYTES of device memory on every
+ *     GPU that loads the library, until the process exits.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (a CUDA runtime query, no allocation); make that first call
+ *     before any stream capture on that device.
+ *   - A launch that would need more workspace than the array holds
+ *     (pa_decode_workspace_size(...) > PA_NO_ALLOC_SCRATCH_BYTES) returns
+ *     PA_ERR_WORKSPACE and launches nothing.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each partial result is written
+ *     before it is read within a call), but calls whose GPU work overlaps in
+ *     time, e.g. on two streams or two host threads, race on it. */
+#define PA_NO_ALLOC_SCRATCH_BYTES (16u << 20)
+PA_API pa_status pa_decode_no_alloc(float *out, const void *q, const void *k_cache,
+                                    const void *v_cache, pa_kv_dtype kv_dtype,
+                                    float k_scale, float v_scale,
+                                    const int32_t *block_tables,
+                                    int max_blocks_per_seq,
+                                    const int32_t *context_lens,
+                                    int max_context_len, int num_seqs,
+                                    int num_q_heads, int num_kv_heads,
+                                    int head_dim, int block_size,
+                                    int num_blocks, float sm_scale,
+                                    int partition_size, void *stream);
+
 /* ------------------------------------------------------- cache writes ---- */
 
 /* Scatter new tokens' K/V into their cache slots: for token t and KV head

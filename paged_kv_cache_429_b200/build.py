@@ -16,7 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpa.so")
 
-SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "pool.cpp")]
+SOURCES = [os.path.join(CSRC, "pa_api.cu"), os.path.join(CSRC, "pa_noalloc.cu"),
+           os.path.join(CSRC, "pool.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)
                   if f.endswith((".cuh", ".h"))] + [os.path.join(INCLUDE, "pa.h")]
 
