@@ -6,30 +6,37 @@
 // physical block block_tables[s][j]; inside a block the 16 token rows are
 // contiguous, between blocks the kernel follows the table.
 //
-// Design (one CTA per (sequence, KV head, partition)):
+// Design. A CTA owns one (sequence, KV head) and a contiguous range of its
+// blocks: the whole context (single-pass), or a chunk of consecutive
+// partitions (split-context, several partitions per CTA so that start-up
+// costs are paid once per chunk):
 //   * a producer warp walks the block table (32 entries per coalesced load)
-//     and, for every logical block, issues two TMA tiled loads (K tile and V
-//     tile of that (block, KV head): 16 x head_dim, contiguous in HBM) into a
-//     ring of shared-memory stages, each guarded by a "full" mbarrier with a
-//     transaction count and an "empty" mbarrier for reuse. The tensor maps
-//     use the 128-byte (64-byte for 64-byte rows) swizzle so that the
-//     ldmatrix reads below are free of bank conflicts. An id outside the pool
-//     is redirected past the tensor's end, where TMA returns zeros.
+//     and, for every logical block in the range, issues two TMA tiled loads
+//     (the K tile and the V tile of that (block, KV head): 16 x head_dim,
+//     contiguous in HBM) into a ring of shared-memory stages, each guarded
+//     by a "full" mbarrier with a transaction count and an "empty" mbarrier
+//     for reuse. The ring runs continuously across partition boundaries.
+//     The tensor maps use the 128-byte (64-byte for 64-byte rows) swizzle so
+//     that the ldmatrix reads below are free of bank conflicts. An id outside
+//     the pool is redirected past the tensor's end, where TMA returns zeros.
 //   * four consumer warps take the stages round-robin. Each warp keeps its
 //     own online-softmax state (running max m, running sum l, unnormalised
 //     output) for all query heads of the KV head (GQA sharing: one K/V tile
 //     serves the whole query group) and computes per 16-token block:
 //       S^T[16 tok][8 heads] = K[16][D] . Q^T[D][8]     (warp MMA m16n8k16)
 //       online softmax over the tokens of each head column (exp2 domain)
-//       O^T[D][8 heads]     += V^T[D][16] . P[16][8]    (warp MMA, P split
-//                              into high and low 16-bit parts so the
-//                              probabilities keep ~16 significant bits)
-//     Tokens past the context length are masked: their scores become -inf
-//     and their V elements are zeroed in registers (the slots may hold NaN).
-//   * at the end the warps' states are merged in shared memory and either
-//     normalised into `out` (single-pass) or written, unnormalised with the
-//     partition's max and sum, to the workspace for the reduce kernel
-//     (split-context).
+//       O^T[D][8 heads]     += V^T[D][16] . P[16][8]    (warp MMA)
+//     For bf16 caches P is split into high and low bf16 parts so that the
+//     probabilities keep ~16 significant bits; for fp8 caches P is one f16.
+//     Tokens past the context length (only in a sequence's last block) are
+//     masked: their scores become -inf and their V elements are zeroed in
+//     registers (those slots may hold NaN).
+//   * at the end of each partition (and of the range) the warps' states are
+//     merged lane by lane (every warp holds the same fragment layout): warps
+//     1-3 hand theirs to warp 0 through shared memory, and warp 0 writes
+//     either the normalised output (single-pass) or the partition's
+//     unnormalised output with its max and sum (split; a second kernel
+//     combines the partitions).
 // fp8 E4M3 caches are widened to f16 exactly (cvt.rn.f16x2.e4m3x2) and use
 // the f16 MMA; q is then scaled per head by a power of two into f16 range
 // (exact), and the power is divided out of the scores.
@@ -63,12 +70,31 @@ struct Geo {
   static constexpr int kBoxBytes = kBoxRow * kBS;
   static constexpr int kTileBytes = kRowBytes * kBS;
   static constexpr int kStageBytes = 2 * kTileBytes;  // K tile + V tile
-  static constexpr int kStagesRaw = 65536 / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
   static constexpr int kKSteps = D / 16;              // MMA k-steps / m-tiles
-  static constexpr int kRingBytes = kStages * kStageBytes;
-  static_assert(kStages % kConsumerWarps == 0, "stages per consumer warp");
   static_assert(kBoxBytes % 512 == 0, "swizzle atom alignment");
+};
+
+// Shared-memory plan of one kernel instance: a 64 KB ring (8 stages of
+// 8 KB for bf16 d128, 16 stages otherwise) and, for the split path, a merge
+// buffer for two warps' per-lane records; 3 CTAs fit per SM either way.
+// Every stage is used by one consumer warp only (stages % warps == 0), so a
+// warp never waits on a stage whose previous use belongs to another warp —
+// an mbarrier parity wait cannot tell a phase from the one two ahead.
+template <int D, bool FP8, int NT, bool CHUNKED>
+struct Plan {
+  using G = Geo<D, FP8>;
+  static constexpr int kStagesRaw = 65536 / G::kStageBytes;
+  static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
+  static constexpr int kRingBytes = kStages * G::kStageBytes;
+  // per-lane merge record: acc[NT][KS] as float4, then (m0, m1, l0, l1)[NT]
+  static constexpr int kLaneFloats = NT * G::kKSteps * 4 + NT * 4;
+  static constexpr int kMergeBytes = 2 * 32 * kLaneFloats * 4;  // warps 2 and 3
+  static constexpr int kMergeOffset = CHUNKED ? kRingBytes : 0;
+  static constexpr int kBarOffset = CHUNKED ? kRingBytes + kMergeBytes : kRingBytes;
+  static constexpr int kSmemBytes = 1024 + kBarOffset + 16 * kStages + 16;
+  static_assert(kStages % kConsumerWarps == 0, "each stage belongs to one consumer warp");
+  static_assert(kStages >= 2 * kConsumerWarps, "two stages per consumer warp");
+  static_assert(CHUNKED || kMergeBytes <= kRingBytes, "merge buffer fits the idle ring");
 };
 
 // Byte offset of (token row r, byte c of the row) inside a swizzled tile.
@@ -100,6 +126,7 @@ struct DecodeParams {
   int group;                    // query heads per KV head
   int num_blocks;
   int partition_blocks;         // blocks per partition; 0 = single-pass
+  int partitions_per_cta;       // split: consecutive partitions per CTA
   int max_partitions;           // P (workspace stride)
   float score_scale;            // sm_scale * log2(e) [* k_scale for fp8]
   float out_scale;              // v_scale for fp8, 1 for bf16
@@ -121,44 +148,343 @@ __device__ __forceinline__ int clamped_len(const int32_t *context_lens, int s,
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
-__device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
+// Named barriers: 1 = the four consumer warps, 2 = consumer warps 0 and 1.
+__device__ __forceinline__ void consumer_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+__device__ __forceinline__ void pair_bar_sync() {
+  asm volatile("bar.sync 2, 64;" ::: "memory");
+}
 
+// Online-softmax state of one consumer warp (per lane: its fragment share).
+template <int D, int NT>
+struct WarpState {
+  float acc[NT][D / 16][4];  // O^T fragments: rows = dims, cols = heads
+  float m[NT][2];            // running max of head columns 2qd, 2qd+1
+  float l[NT][2];            // running sum (this lane's tokens only)
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt)
+        acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
+    }
+  }
+};
+
+// One 16-token block for one consumer warp. TAIL: the block holds the end of
+// the context (`valid` < 16 tokens are real).
+template <int D, bool FP8, int NT, bool TAIL>
+__device__ __forceinline__ void attend_block(uint32_t kt, uint32_t vt, int valid, int lane,
+                                             const uint32_t (&qf)[NT][D / 16][2],
+                                             const float (&cs)[NT][2],
+                                             WarpState<D, NT> &ws) {
+  constexpr int KS = D / 16;
+  const int mi = lane >> 3;    // ldmatrix: lane supplies a row of matrix mi
+  const int mrow = lane & 7;
+  const int gq = lane >> 2;    // MMA group id: token row / head column
+  const int qd = lane & 3;     // thread in group
+
+  // ---- scores S^T = K . Q^T  (two accumulator chains for ILP)
+  float sc[NT][2][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) sc[nt][c][0] = sc[nt][c][1] = sc[nt][c][2] = sc[nt][c][3] = 0.f;
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * ks + (mi >> 1) * 16), a0, a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        mma_16816<false>(sc[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < KS / 2; ++kk) {
+      // r0/r1: rows 0-7 / 8-15, dims [32kk, 32kk+16); r2/r3: the next 16 dims.
+      // Each register holds dims 4qd..4qd+3 of its row.
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * kk + (mi >> 1) * 16), r0, r1, r2, r3);
+      uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+      e4m3x4_to_f16x2x2(r0, a0, a2);
+      e4m3x4_to_f16x2x2(r1, a1, a3);
+      e4m3x4_to_f16x2x2(r2, c0, c2);
+      e4m3x4_to_f16x2x2(r3, c1, c3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816<true>(sc[nt][0], a0, a1, a2, a3, qf[nt][2 * kk][0], qf[nt][2 * kk][1]);
+        mma_16816<true>(sc[nt][1], c0, c1, c2, c3, qf[nt][2 * kk + 1][0], qf[nt][2 * kk + 1][1]);
+      }
+    }
+  }
+
+  // ---- online softmax per head column
+  uint32_t pb_hi[NT][2], pb_lo[NT][2];
+  float alpha[NT][2];
+  bool rescale = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float z0 = (sc[nt][0][0] + sc[nt][1][0]) * cs[nt][0];  // token gq,   head 2qd
+    float z1 = (sc[nt][0][1] + sc[nt][1][1]) * cs[nt][1];  // token gq,   head 2qd+1
+    float z2 = (sc[nt][0][2] + sc[nt][1][2]) * cs[nt][0];  // token gq+8, head 2qd
+    float z3 = (sc[nt][0][3] + sc[nt][1][3]) * cs[nt][1];  // token gq+8, head 2qd+1
+    if constexpr (TAIL) {
+      if (gq >= valid) z0 = z1 = -INFINITY;
+      if (gq + 8 >= valid) z2 = z3 = -INFINITY;
+    }
+    float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(ws.m[nt][0], mx0);
+    const float mn1 = fmaxf(ws.m[nt][1], mx1);
+    alpha[nt][0] = exp2f(ws.m[nt][0] - mn0);
+    alpha[nt][1] = exp2f(ws.m[nt][1] - mn1);
+    rescale |= (ws.m[nt][0] != mn0) || (ws.m[nt][1] != mn1);
+    ws.m[nt][0] = mn0;
+    ws.m[nt][1] = mn1;
+    const float p0 = exp2f(z0 - mn0), p1 = exp2f(z1 - mn1);
+    const float p2 = exp2f(z2 - mn0), p3 = exp2f(z3 - mn1);
+    ws.l[nt][0] = ws.l[nt][0] * alpha[nt][0] + (p0 + p2);
+    ws.l[nt][1] = ws.l[nt][1] * alpha[nt][1] + (p1 + p3);
+    // P as the B operand (rows = tokens, cols = heads): build the two 8x8
+    // tiles (tokens 0-7 / 8-15) x heads in accumulator layout, transpose each
+    const uint32_t h01 = pack2<FP8>(p0, p1), h23 = pack2<FP8>(p2, p3);
+    pb_hi[nt][0] = movmatrix_trans(h01);
+    pb_hi[nt][1] = movmatrix_trans(h23);
+    if constexpr (!FP8) {
+      float u0, u1, u2, u3;
+      unpack2<false>(h01, u0, u1);
+      unpack2<false>(h23, u2, u3);
+      pb_lo[nt][0] = movmatrix_trans(pack2<false>(p0 - u0, p1 - u1));
+      pb_lo[nt][1] = movmatrix_trans(pack2<false>(p2 - u2, p3 - u3));
+    }
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        ws.acc[nt][mt][0] *= alpha[nt][0];
+        ws.acc[nt][mt][1] *= alpha[nt][1];
+        ws.acc[nt][mt][2] *= alpha[nt][0];
+        ws.acc[nt][mt][3] *= alpha[nt][1];
+      }
+  }
+
+  // ---- O^T += V^T . P ; V of tokens >= valid is zeroed (tail block only)
+  uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+  if constexpr (TAIL) {
+    mlo = (2 * qd < valid ? 0x0000ffffu : 0u) | (2 * qd + 1 < valid ? 0xffff0000u : 0u);
+    mhi = (2 * qd + 8 < valid ? 0x0000ffffu : 0u) | (2 * qd + 9 < valid ? 0xffff0000u : 0u);
+  }
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(vt + swz<D, FP8>((mi >> 1) * 8 + mrow, 32 * mt + (mi & 1) * 16), a0, a1, a2, a3);
+      if constexpr (TAIL) {
+        a0 &= mlo;
+        a1 &= mlo;
+        a2 &= mhi;
+        a3 &= mhi;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
+        mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_lo[nt][0], pb_lo[nt][1]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int cc = 0; cc < KS / 2; ++cc) {
+      // r0/r1: tokens 0-7 / 8-15 of dims [32cc, 32cc+16); r2/r3: next 16
+      // dims. Bytes of r: (t,2g) (t,2g+1) (t+1,2g) (t+1,2g+1) with
+      // t = 2qd, g = gq; regroup into token pairs per dim, then widen.
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_trans(vt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * cc + (mi >> 1) * 16), r0, r1, r2, r3);
+      uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+      e4m3x4_to_f16x2x2(prmt(r0, 0x3120), a0, a1);
+      e4m3x4_to_f16x2x2(prmt(r1, 0x3120), a2, a3);
+      e4m3x4_to_f16x2x2(prmt(r2, 0x3120), c0, c1);
+      e4m3x4_to_f16x2x2(prmt(r3, 0x3120), c2, c3);
+      if constexpr (TAIL) {
+        a0 &= mlo;
+        a1 &= mlo;
+        a2 &= mhi;
+        a3 &= mhi;
+        c0 &= mlo;
+        c1 &= mlo;
+        c2 &= mhi;
+        c3 &= mhi;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816<true>(ws.acc[nt][2 * cc], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
+        mma_16816<true>(ws.acc[nt][2 * cc + 1], c0, c1, c2, c3, pb_hi[nt][0], pb_hi[nt][1]);
+      }
+    }
+  }
+}
+
+template <int D, int NT>
+__device__ __forceinline__ void store_record(const WarpState<D, NT> &ws, float *rec) {
+  float4 *r = reinterpret_cast<float4 *>(rec);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+      r[nt * (D / 16) + mt] = make_float4(ws.acc[nt][mt][0], ws.acc[nt][mt][1],
+                                          ws.acc[nt][mt][2], ws.acc[nt][mt][3]);
+    r[NT * (D / 16) + nt] = make_float4(ws.m[nt][0], ws.m[nt][1], ws.l[nt][0], ws.l[nt][1]);
+  }
+}
+
+// Fold another warp's record (same lane, same fragment layout) into ws.
+template <int D, int NT>
+__device__ __forceinline__ void combine_record(WarpState<D, NT> &ws, const float *rec) {
+  const float4 *r = reinterpret_cast<const float4 *>(rec);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float4 ml = r[NT * (D / 16) + nt];
+    const float mo[2] = {ml.x, ml.y}, lo[2] = {ml.z, ml.w};
+    float wa[2], wb[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const float M = fmaxf(ws.m[nt][c], mo[c]);
+      wa[c] = (M == -INFINITY) ? 0.f : exp2f(ws.m[nt][c] - M);
+      wb[c] = (M == -INFINITY) ? 0.f : exp2f(mo[c] - M);
+      ws.l[nt][c] = wa[c] * ws.l[nt][c] + wb[c] * lo[c];
+      ws.m[nt][c] = M;
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const float4 o = r[nt * (D / 16) + mt];
+      ws.acc[nt][mt][0] = wa[0] * ws.acc[nt][mt][0] + wb[0] * o.x;
+      ws.acc[nt][mt][1] = wa[1] * ws.acc[nt][mt][1] + wb[1] * o.y;
+      ws.acc[nt][mt][2] = wa[0] * ws.acc[nt][mt][2] + wb[0] * o.z;
+      ws.acc[nt][mt][3] = wa[1] * ws.acc[nt][mt][3] + wb[1] * o.w;
+    }
+  }
+}
+
+// Merge the four consumer warps' states lane by lane (every warp holds the
+// same fragment layout) as a two-level tree — warps 2, 3 into 0, 1, then 1
+// into 0 — through `mbuf` (two per-lane records), and let warp 0 write the
+// result: out[] (single-pass) or one partition's workspace row (split).
 template <int D, bool FP8, int NT>
+__device__ __forceinline__ void merge_and_write(WarpState<D, NT> &ws, float *mbuf, int warp,
+                                                int lane, const DecodeParams &p, int s, int h,
+                                                int partition, bool split) {
+  constexpr int KS = D / 16;
+  constexpr int LF = NT * KS * 4 + NT * 4;
+  const int gq = lane >> 2;
+  const int qd = lane & 3;
+  // l so far is per lane (its two token rows); total per head column
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) ws.l[nt][c] += __shfl_xor_sync(0xffffffffu, ws.l[nt][c], o);
+  if (warp >= 2) store_record<D, NT>(ws, mbuf + ((warp - 2) * 32 + lane) * LF);
+  consumer_bar_sync();
+  if (warp >= 2) return;
+  combine_record<D, NT>(ws, mbuf + (warp * 32 + lane) * LF);
+  pair_bar_sync();  // warps 0 and 1 have read their records
+  if (warp == 1) store_record<D, NT>(ws, mbuf + lane * LF);
+  pair_bar_sync();
+  if (warp == 1) return;
+  combine_record<D, NT>(ws, mbuf + lane * LF);
+
+  const int group = p.group;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int n0 = nt * 8 + 2 * qd;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int n = n0 + c;
+      if (n >= group) continue;
+      const int hq = h * group + n;
+      const float L = ws.l[nt][c];
+      float *dst;
+      float scale;
+      if (!split) {
+        dst = p.out + (static_cast<int64_t>(s) * p.num_q_heads + hq) * D;
+        scale = (L > 0.f) ? p.out_scale / L : 0.f;
+      } else {
+        const int64_t row = (static_cast<int64_t>(s) * p.num_q_heads + hq) * p.max_partitions + partition;
+        dst = p.ws_o + row * D;
+        scale = p.out_scale;
+        if (gq == 0) {
+          p.ws_m[row] = ws.m[nt][c];
+          p.ws_l[row] = L;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        int d0, d1;
+        if constexpr (!FP8) {
+          d0 = 16 * mt + gq;
+          d1 = d0 + 8;
+        } else {
+          d0 = 16 * mt + 2 * gq;
+          d1 = d0 + 1;
+        }
+        dst[d0] = ws.acc[nt][mt][c] * scale;
+        dst[d1] = ws.acc[nt][mt][2 + c] * scale;
+      }
+    }
+  }
+}
+
+template <int D, bool FP8, int NT, bool CHUNKED>
 __global__ void __launch_bounds__(kDecodeThreads)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v,
                         const DecodeParams p) {
   using G = Geo<D, FP8>;
-  constexpr int NS = G::kStages;
+  using PL = Plan<D, FP8, NT, CHUNKED>;
+  constexpr int NS = PL::kStages;
   constexpr int KS = G::kKSteps;
-  constexpr int HN = NT * 8;  // padded query heads handled by this CTA
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t ring = (raw_u32 + 1023u) & ~1023u;
-  uint8_t *ring_ptr = smem_raw + (ring - raw_u32);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ring_ptr + G::kRingBytes);
-  const uint32_t full0 = smem_u32(bars);           // full[i]  at full0 + 8i
-  const uint32_t empty0 = full0 + 8u * NS;         // empty[i] at empty0 + 8i
+  uint8_t *base_ptr = smem_raw + (ring - raw_u32);
+  float *mbuf = reinterpret_cast<float *>(base_ptr + PL::kMergeOffset);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base_ptr + PL::kBarOffset);
+  const uint32_t full0 = smem_u32(bars);    // full[i]  at full0 + 8i
+  const uint32_t empty0 = full0 + 8u * NS;  // empty[i] at empty0 + 8i
   volatile int *s_abort = reinterpret_cast<volatile int *>(bars + 2 * NS);
 
-  const int part = blockIdx.x;
+  const int chunk = blockIdx.x;
   const int h = blockIdx.y;
   const int s = blockIdx.z;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   bool bad_len;
-  const int L = clamped_len(p.context_lens, s, p.max_context_len,
-                            p.max_blocks_per_seq, &bad_len);
+  const int L = clamped_len(p.context_lens, s, p.max_context_len, p.max_blocks_per_seq, &bad_len);
   const int nb_seq = (L + kBS - 1) / kBS;
-  int j0 = 0, j1 = nb_seq;
-  if (p.partition_blocks > 0) {
-    j0 = part * p.partition_blocks;
-    j1 = min(nb_seq, j0 + p.partition_blocks);
-    if (j0 >= j1) return;  // partition past this sequence's end: no output
+  // block range [j0, j1) of this CTA; split: partitions [pc0, pc0 + npart)
+  int j0 = 0, j1 = nb_seq, pc0 = 0, npart = 1;
+  const int pb = p.partition_blocks;
+  if (CHUNKED) {
+    pc0 = chunk * p.partitions_per_cta;
+    j0 = pc0 * pb;
+    if (j0 >= nb_seq) return;  // chunk past this sequence's end: no output
+    j1 = min(nb_seq, j0 + p.partitions_per_cta * pb);
+    npart = (j1 - j0 + pb - 1) / pb;
   }
-  if (bad_len && threadIdx.x == 0 && part == 0) raise_error(kErrContextClamp);
+  if (bad_len && threadIdx.x == 0 && chunk == 0) raise_error(kErrContextClamp);
   const int nblk = j1 - j0;
 
   if (threadIdx.x == 0) {
@@ -193,8 +519,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
           if (it >= NS) {
             if (*s_abort) {
               ok = false;
-            } else if (!mbar_wait_bounded(empty0 + 8u * st, ((it / NS) - 1) & 1,
-                                          kWaitLimitNs)) {
+            } else if (!mbar_wait_bounded(empty0 + 8u * st, ((it / NS) - 1) & 1, kWaitLimitNs)) {
               ok = false;
               *s_abort = 1;
               raise_error(kErrWaitTimeout);
@@ -231,308 +556,111 @@ __global__ void __launch_bounds__(kDecodeThreads)
       for (int it = max(0, issued - NS); it < issued; ++it)
         mbar_wait_bounded(full0 + 8u * (it % NS), (it / NS) & 1, kWaitLimitNs);
     }
+    if (!CHUNKED) __syncthreads();  // single-pass: the merge reuses the ring
+    return;
   }
 
   // ------------------------------------------------------------ consumers
-  float acc[NT][KS][4];
-  float m_run[NT][2], l_run[NT][2];
-  const int gq = lane >> 2;  // MMA group id: token row / head column index
-  const int qd = lane & 3;   // thread in group
-  if (warp < kConsumerWarps) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      m_run[nt][0] = m_run[nt][1] = -INFINITY;
-      l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
-        acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
-    }
+  const int gq = lane >> 2;
+  const int qd = lane & 3;
+  WarpState<D, NT> ws;
+  ws.reset();
 
-    // Q^T fragments (B operand): head column gq, k-slots by thread qd.
-    uint32_t qf[NT][KS][2];
-    float col_scale[NT][2];
+  // Q^T fragments (B operand): head column gq, k-slots by thread qd.
+  uint32_t qf[NT][KS][2];
+  float cs[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int n = nt * 8 + gq;
-      const bool live = n < p.group;
-      const uint16_t *qrow = p.q + (static_cast<int64_t>(s) * p.num_q_heads +
-                                    h * p.group + (live ? n : 0)) * D;
-      if constexpr (!FP8) {
+  for (int nt = 0; nt < NT; ++nt) {
+    const int n = nt * 8 + gq;
+    const bool live = n < p.group;
+    const uint16_t *qrow = p.q + (static_cast<int64_t>(s) * p.num_q_heads + h * p.group + (live ? n : 0)) * D;
+    if constexpr (!FP8) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qf[nt][ks][0] = live ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * qd) : 0u;
-          qf[nt][ks][1] = live ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * qd) : 0u;
-        }
-        col_scale[nt][0] = col_scale[nt][1] = p.score_scale;
-      } else {
-        // k-slot order matching the fp8 K fragments: slots (2qd, 2qd+1) ->
-        // dims (4qd, 4qd+1), slots (2qd+8, 2qd+9) -> dims (4qd+2, 4qd+3).
-        float v[KS][4];
-        float amax = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint2 w = live ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * qd)
-                         : make_uint2(0u, 0u);
-          v[ks][0] = __uint_as_float(w.x << 16);
-          v[ks][1] = __uint_as_float(w.x & 0xFFFF0000u);
-          v[ks][2] = __uint_as_float(w.y << 16);
-          v[ks][3] = __uint_as_float(w.y & 0xFFFF0000u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[ks][e]));
-        }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        // power of two 2^e with amax * 2^e in [2^14, 2^15): exact in f16
-        int ex = 0;
-        if (amax > 0.f && amax <= 3.0e38f) {
-          int E;
-          frexpf(amax, &E);
-          ex = 15 - E;
-          ex = ex > 126 ? 126 : (ex < -126 ? -126 : ex);
-        }
-        const float up = __int_as_float((127 + ex) << 23);
-        const float down = __int_as_float((127 - ex) << 23);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qf[nt][ks][0] = pack2<true>(v[ks][0] * up, v[ks][1] * up);
-          qf[nt][ks][1] = pack2<true>(v[ks][2] * up, v[ks][3] * up);
-        }
-        // this thread's score columns are heads 2qd and 2qd+1 of the tile
-        col_scale[nt][0] = p.score_scale * __shfl_sync(0xffffffffu, down, 8 * qd);
-        col_scale[nt][1] = p.score_scale * __shfl_sync(0xffffffffu, down, 8 * qd + 4);
+      for (int ks = 0; ks < KS; ++ks) {
+        qf[nt][ks][0] = live ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 2 * qd) : 0u;
+        qf[nt][ks][1] = live ? *reinterpret_cast<const uint32_t *>(qrow + 16 * ks + 8 + 2 * qd) : 0u;
       }
-    }
-
-    // ldmatrix row addresses: lane supplies row (lane & 7) of matrix lane >> 3
-    const int mi = lane >> 3;
-    const int mrow = lane & 7;
-    bool aborted = false;
-
-    for (int it = warp; it < nblk; it += kConsumerWarps) {
-      const int st = it % NS;
-      const bool got = mbar_wait_bounded(full0 + 8u * st, (it / NS) & 1, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, got)) {
-        aborted = true;
-        break;
-      }
-      const uint32_t kt = ring + st * G::kStageBytes;
-      const uint32_t vt = kt + G::kTileBytes;
-      const int valid = min(kBS, L - (j0 + it) * kBS);
-
-      // ---- scores S^T = K . Q^T  (two accumulator chains for ILP)
-      float sc[NT][2][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          sc[nt][c][0] = sc[nt][c][1] = sc[nt][c][2] = sc[nt][c][3] = 0.f;
-      if constexpr (!FP8) {
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * ks + (mi >> 1) * 16), a0, a1, a2, a3);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_16816<false>(sc[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-        }
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < KS / 2; ++kk) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * kk + (mi >> 1) * 16), r0, r1, r2, r3);
-          const uint32_t a00 = e4m3x2_to_f16x2(r0), a02 = e4m3x2_to_f16x2(r0 >> 16);
-          const uint32_t a01 = e4m3x2_to_f16x2(r1), a03 = e4m3x2_to_f16x2(r1 >> 16);
-          const uint32_t a10 = e4m3x2_to_f16x2(r2), a12 = e4m3x2_to_f16x2(r2 >> 16);
-          const uint32_t a11 = e4m3x2_to_f16x2(r3), a13 = e4m3x2_to_f16x2(r3 >> 16);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<true>(sc[nt][0], a00, a01, a02, a03, qf[nt][2 * kk][0], qf[nt][2 * kk][1]);
-            mma_16816<true>(sc[nt][1], a10, a11, a12, a13, qf[nt][2 * kk + 1][0], qf[nt][2 * kk + 1][1]);
-          }
-        }
-      }
-
-      // ---- online softmax per head column (exp2 domain)
-      uint32_t pb_hi[NT][2], pb_lo[NT][2];
-      float alpha[NT][2];
-      bool rescale = false;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float z[4];
-        z[0] = (sc[nt][0][0] + sc[nt][1][0]) * col_scale[nt][0];  // tok gq,   head 2qd
-        z[1] = (sc[nt][0][1] + sc[nt][1][1]) * col_scale[nt][1];  // tok gq,   head 2qd+1
-        z[2] = (sc[nt][0][2] + sc[nt][1][2]) * col_scale[nt][0];  // tok gq+8, head 2qd
-        z[3] = (sc[nt][0][3] + sc[nt][1][3]) * col_scale[nt][1];  // tok gq+8, head 2qd+1
-        if (gq >= valid) z[0] = z[1] = -INFINITY;
-        if (gq + 8 >= valid) z[2] = z[3] = -INFINITY;
-        float mx0 = fmaxf(z[0], z[2]), mx1 = fmaxf(z[1], z[3]);
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        const float mn0 = fmaxf(m_run[nt][0], mx0);
-        const float mn1 = fmaxf(m_run[nt][1], mx1);
-        alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-        alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-        rescale |= (alpha[nt][0] != 1.f) || (alpha[nt][1] != 1.f);
-        m_run[nt][0] = mn0;
-        m_run[nt][1] = mn1;
-        const float p0 = fast_exp2(z[0] - mn0), p1 = fast_exp2(z[1] - mn1);
-        const float p2 = fast_exp2(z[2] - mn0), p3 = fast_exp2(z[3] - mn1);
-        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (p0 + p2);
-        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (p1 + p3);
-        // P as the B operand: rows = tokens, cols = heads. Build the 8x8
-        // tiles (tokens 0-7 / 8-15) x heads in accumulator layout, then
-        // transpose each in registers.
-        const uint32_t h01 = pack2<FP8>(p0, p1), h23 = pack2<FP8>(p2, p3);
-        float u0, u1, u2, u3;
-        unpack2<FP8>(h01, u0, u1);
-        unpack2<FP8>(h23, u2, u3);
-        const uint32_t l01 = pack2<FP8>(p0 - u0, p1 - u1), l23 = pack2<FP8>(p2 - u2, p3 - u3);
-        pb_hi[nt][0] = movmatrix_trans(h01);
-        pb_hi[nt][1] = movmatrix_trans(h23);
-        pb_lo[nt][0] = movmatrix_trans(l01);
-        pb_lo[nt][1] = movmatrix_trans(l23);
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            acc[nt][mt][0] *= alpha[nt][0];
-            acc[nt][mt][1] *= alpha[nt][1];
-            acc[nt][mt][2] *= alpha[nt][0];
-            acc[nt][mt][3] *= alpha[nt][1];
-          }
-      }
-
-      // ---- O^T += V^T . P ; V elements of tokens >= valid are zeroed
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-      if (valid < kBS) {
-        mlo = (2 * qd < valid ? 0x0000ffffu : 0u) | (2 * qd + 1 < valid ? 0xffff0000u : 0u);
-        mhi = (2 * qd + 8 < valid ? 0x0000ffffu : 0u) | (2 * qd + 9 < valid ? 0xffff0000u : 0u);
-      }
-      if constexpr (!FP8) {
-#pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(vt + swz<D, FP8>((mi >> 1) * 8 + mrow, 32 * mt + (mi & 1) * 16), a0, a1, a2, a3);
-          a0 &= mlo;
-          a1 &= mlo;
-          a2 &= mhi;
-          a3 &= mhi;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<false>(acc[nt][mt], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
-            mma_16816<false>(acc[nt][mt], a0, a1, a2, a3, pb_lo[nt][0], pb_lo[nt][1]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < KS / 2; ++cc) {
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4_trans(vt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * cc + (mi >> 1) * 16), r0, r1, r2, r3);
-          // r0/r1: tokens 0-7 / 8-15 of dims [32cc, 32cc+16); r2/r3: next 16
-          // dims. Bytes of r: (t,2g) (t,2g+1) (t+1,2g) (t+1,2g+1) with
-          // t = 2qd; regroup into token pairs per dim, then widen.
-          const uint32_t t0 = prmt(r0, 0x3120), t1 = prmt(r1, 0x3120);
-          const uint32_t t2 = prmt(r2, 0x3120), t3 = prmt(r3, 0x3120);
-          const uint32_t a0 = e4m3x2_to_f16x2(t0) & mlo, a1 = e4m3x2_to_f16x2(t0 >> 16) & mlo;
-          const uint32_t a2 = e4m3x2_to_f16x2(t1) & mhi, a3 = e4m3x2_to_f16x2(t1 >> 16) & mhi;
-          const uint32_t c0 = e4m3x2_to_f16x2(t2) & mlo, c1 = e4m3x2_to_f16x2(t2 >> 16) & mlo;
-          const uint32_t c2 = e4m3x2_to_f16x2(t3) & mhi, c3 = e4m3x2_to_f16x2(t3 >> 16) & mhi;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<true>(acc[nt][2 * cc], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
-            mma_16816<true>(acc[nt][2 * cc], a0, a1, a2, a3, pb_lo[nt][0], pb_lo[nt][1]);
-            mma_16816<true>(acc[nt][2 * cc + 1], c0, c1, c2, c3, pb_hi[nt][0], pb_hi[nt][1]);
-            mma_16816<true>(acc[nt][2 * cc + 1], c0, c1, c2, c3, pb_lo[nt][0], pb_lo[nt][1]);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8u * st);
-    }
-    if (aborted && lane == 0) {
-      *s_abort = 1;
-      raise_error(kErrWaitTimeout);
-    }
-    // total l per head column: sum over the 8 token-row groups
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1)
-          l_run[nt][c] += __shfl_xor_sync(0xffffffffu, l_run[nt][c], o);
-  }
-  __syncthreads();  // ring is idle from here on: reuse it for the merge
-
-  // ------------------------------------------------- merge the warps' states
-  float *mg_o = reinterpret_cast<float *>(ring_ptr);            // [W][HN][D]
-  float *mg_m = mg_o + kConsumerWarps * HN * D;                 // [W][HN]
-  float *mg_l = mg_m + kConsumerWarps * HN;                     // [W][HN]
-  if (warp < kConsumerWarps) {
-    float *ow = mg_o + warp * HN * D;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int n0 = nt * 8 + 2 * qd;
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        int d0, d1;
-        if constexpr (!FP8) {
-          d0 = 16 * mt + gq;
-          d1 = d0 + 8;
-        } else {
-          d0 = 16 * mt + 2 * gq;
-          d1 = d0 + 1;
-        }
-        ow[n0 * D + d0] = acc[nt][mt][0];
-        ow[(n0 + 1) * D + d0] = acc[nt][mt][1];
-        ow[n0 * D + d1] = acc[nt][mt][2];
-        ow[(n0 + 1) * D + d1] = acc[nt][mt][3];
-      }
-      if (gq == 0) {
-        mg_m[warp * HN + n0] = m_run[nt][0];
-        mg_m[warp * HN + n0 + 1] = m_run[nt][1];
-        mg_l[warp * HN + n0] = l_run[nt][0];
-        mg_l[warp * HN + n0 + 1] = l_run[nt][1];
-      }
-    }
-  }
-  __syncthreads();
-
-  const int group = p.group;
-  for (int idx = threadIdx.x; idx < group * D; idx += kDecodeThreads) {
-    const int n = idx / D;
-    const int d = idx - n * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mg_m[w * HN + n]);
-    float o = 0.f, l = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float wt = fast_exp2(mg_m[w * HN + n] - M);
-        o += wt * mg_o[(w * HN + n) * D + d];
-        l += wt * mg_l[w * HN + n];
-      }
-    }
-    const int hq = h * group + n;
-    if (p.partition_blocks == 0) {
-      p.out[(static_cast<int64_t>(s) * p.num_q_heads + hq) * D + d] =
-          (l > 0.f) ? o * p.out_scale / l : 0.f;
+      cs[nt][0] = cs[nt][1] = p.score_scale;
     } else {
-      const int64_t row = (static_cast<int64_t>(s) * p.num_q_heads + hq) * p.max_partitions + part;
-      p.ws_o[row * D + d] = o * p.out_scale;
-      if (d == 0) {
-        p.ws_m[row] = M;
-        p.ws_l[row] = l;
+      // k-slot order matching the fp8 K fragments: slots (2qd, 2qd+1) ->
+      // dims (4qd, 4qd+1), slots (2qd+8, 2qd+9) -> dims (4qd+2, 4qd+3).
+      float v[KS][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint2 w = live ? *reinterpret_cast<const uint2 *>(qrow + 16 * ks + 4 * qd) : make_uint2(0u, 0u);
+        v[ks][0] = __uint_as_float(w.x << 16);
+        v[ks][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        v[ks][2] = __uint_as_float(w.y << 16);
+        v[ks][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[ks][e]));
       }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // power of two 2^e with amax * 2^e in [2^14, 2^15): exact in f16
+      int ex = 0;
+      if (amax > 0.f && amax <= 3.0e38f) {
+        int E;
+        frexpf(amax, &E);
+        ex = 15 - E;
+        ex = ex > 126 ? 126 : (ex < -126 ? -126 : ex);
+      }
+      const float up = __int_as_float((127 + ex) << 23);
+      const float down = __int_as_float((127 - ex) << 23);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        qf[nt][ks][0] = pack2<true>(v[ks][0] * up, v[ks][1] * up);
+        qf[nt][ks][1] = pack2<true>(v[ks][2] * up, v[ks][3] * up);
+      }
+      // this thread's score columns are heads 2qd and 2qd+1 of the tile
+      cs[nt][0] = p.score_scale * __shfl_sync(0xffffffffu, down, 8 * qd);
+      cs[nt][1] = p.score_scale * __shfl_sync(0xffffffffu, down, 8 * qd + 4);
+    }
+  }
+
+  // Blocks of this warp: it = warp, warp + 4, ... over [0, nblk). Split
+  // ranges are whole partitions of pb blocks, pb a multiple of 4, so every
+  // warp crosses a partition boundary at the same iteration.
+  bool aborted = false;
+  int it = warp;
+  for (int pi = 0; pi < npart; ++pi) {
+    const int it_end = CHUNKED ? min(nblk, (pi + 1) * pb) : nblk;
+    for (; it < it_end; it += kConsumerWarps) {
+      if (!aborted) {
+        const int st = it % NS;
+        const bool got = mbar_wait_bounded(full0 + 8u * st, (it / NS) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          aborted = true;
+          if (lane == 0) {
+            *s_abort = 1;
+            raise_error(kErrWaitTimeout);
+          }
+          continue;
+        }
+        const uint32_t kt = ring + st * G::kStageBytes;
+        const uint32_t vt = kt + G::kTileBytes;
+        const int valid = L - (j0 + it) * kBS;
+        if (valid >= kBS)
+          attend_block<D, FP8, NT, false>(kt, vt, kBS, lane, qf, cs, ws);
+        else
+          attend_block<D, FP8, NT, true>(kt, vt, valid, lane, qf, cs, ws);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8u * st);
+      }
+    }
+    if (CHUNKED) {
+      consumer_bar_sync();  // the previous partition's merge has read mbuf
+      merge_and_write<D, FP8, NT>(ws, mbuf, warp, lane, p, s, h, pc0 + pi, true);
+      ws.reset();
+    } else {
+      __syncthreads();  // all loads consumed: the ring is idle
+      merge_and_write<D, FP8, NT>(ws, reinterpret_cast<float *>(base_ptr), warp, lane, p, s, h, 0,
+                                  false);
     }
   }
 }
+
 
 // Combine the partitions of one (sequence, query head):
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.

@@ -73,12 +73,6 @@ bool make_cache_tmap(CUtensorMap *map, const void *base, int rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, int NT>
-size_t decode_smem_bytes() {
-  using G = Geo<D, FP8>;
-  return 1024 + G::kRingBytes + 16 * G::kStages + 16;
-}
-
 template <typename Kern>
 bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int dev) {
   const uint64_t bit = 1ull << (dev & 63);
@@ -90,7 +84,7 @@ bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int 
   return true;
 }
 
-template <int D, bool FP8, int NT>
+template <int D, bool FP8, int NT, bool CHUNKED>
 pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
                         const DecodeParams &p, int num_seqs, int grid_x,
                         cudaStream_t stream, int dev) {
@@ -98,9 +92,9 @@ pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
   if (!make_cache_tmap<D, FP8>(&tk, k_cache, rows) ||
       !make_cache_tmap<D, FP8>(&tv, v_cache, rows))
     return PA_ERR_CUDA;
-  auto kern = pa::paged_decode_kernel<D, FP8, NT>;
+  auto kern = pa::paged_decode_kernel<D, FP8, NT, CHUNKED>;
   static std::atomic<uint64_t> attr_done{0};
-  const size_t smem = decode_smem_bytes<D, FP8, NT>();
+  const size_t smem = pa::Plan<D, FP8, NT, CHUNKED>::kSmemBytes;
   if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
   dim3 grid(grid_x, p.num_kv_heads, num_seqs);
   kern<<<grid, pa::kDecodeThreads, smem, stream>>>(tk, tv, p);
@@ -121,10 +115,29 @@ pa_status launch_reduce(const ReduceParams &r, int num_seqs, cudaStream_t stream
 }
 
 template <int D, bool FP8>
-pa_status dispatch_nt(int nt, const void *kc, const void *vc, int rows, const DecodeParams &p,
-                      int num_seqs, int grid_x, cudaStream_t st, int dev) {
-  return nt == 1 ? launch_decode<D, FP8, 1>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
-                 : launch_decode<D, FP8, 2>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+pa_status dispatch_nt(int nt, bool chunked, const void *kc, const void *vc, int rows,
+                      const DecodeParams &p, int num_seqs, int grid_x, cudaStream_t st,
+                      int dev) {
+  if (chunked)
+    return nt == 1 ? launch_decode<D, FP8, 1, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                   : launch_decode<D, FP8, 2, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+  return nt == 1 ? launch_decode<D, FP8, 1, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                 : launch_decode<D, FP8, 2, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+}
+
+// Consecutive partitions per CTA in the split path: about 1 MB of K/V per
+// CTA, while keeping at least four CTAs per SM in the grid. Chunks need
+// partitions of a multiple of 4 blocks (one per consumer warp per round).
+int partitions_per_cta(int64_t units, int64_t P, int psize, int num_kv_heads_unused,
+                       int head_dim, int eb, int sms) {
+  (void)num_kv_heads_unused;
+  const int pb = psize / pa::kBS;
+  if (pb % pa::kConsumerWarps != 0) return 1;
+  const int64_t part_bytes = static_cast<int64_t>(psize) * head_dim * eb * 2;
+  int64_t ppc = std::max<int64_t>(1, (int64_t{1} << 20) / std::max<int64_t>(part_bytes, 1));
+  ppc = std::min<int64_t>(ppc, P);
+  while (ppc > 1 && units * ((P + ppc - 1) / ppc) < 4LL * sms) ppc = (ppc + 1) / 2;
+  return static_cast<int>(ppc);
 }
 
 size_t workspace_bytes_for(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
@@ -261,18 +274,25 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
     p.ws_l = reinterpret_cast<float *>(ws + o_bytes + m_bytes);
     p.partition_blocks = psize / pa::kBS;
     p.max_partitions = static_cast<int>(P);
-    grid_x = static_cast<int>(P);
+    p.partitions_per_cta = partitions_per_cta(static_cast<int64_t>(num_seqs) * num_kv_heads, P,
+                                              psize, num_kv_heads, head_dim,
+                                              kv_dtype == PA_KV_BF16 ? 2 : 1,
+                                              device_sm_count(dev));
+    grid_x = static_cast<int>((P + p.partitions_per_cta - 1) / p.partitions_per_cta);
   }
 
   const int nt = group <= 8 ? 1 : 2;
+  const bool chunked = psize > 0;
   const int rows = static_cast<int>(rows64);
   pa_status rc;
   if (kv_dtype == PA_KV_BF16)
-    rc = head_dim == 128 ? dispatch_nt<128, false>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
-                         : dispatch_nt<64, false>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
+    rc = head_dim == 128
+             ? dispatch_nt<128, false>(nt, chunked, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
+             : dispatch_nt<64, false>(nt, chunked, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
   else
-    rc = head_dim == 128 ? dispatch_nt<128, true>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
-                         : dispatch_nt<64, true>(nt, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
+    rc = head_dim == 128
+             ? dispatch_nt<128, true>(nt, chunked, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)
+             : dispatch_nt<64, true>(nt, chunked, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev);
   if (rc != PA_OK || psize == 0) return rc;
 
   ReduceParams r{};

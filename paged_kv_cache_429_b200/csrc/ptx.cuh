@@ -136,16 +136,14 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0,
 
 // ------------------------------------------------------------ conversions
 
-// Two E4M3 codes (low 16 bits of x, element 0 in the low byte) -> f16x2.
+// Four E4M3 codes (bytes 0..3 of x) -> two f16x2: lo = (b0, b1), hi = (b2, b3).
 // Exact: every E4M3 value is an f16 normal number or zero.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
-  uint32_t y;
-  asm volatile(
-      "{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
-      : "=r"(y)
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t &lo, uint32_t &hi) {
+  asm(
+      "{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
       : "r"(x));
-  return y;
 }
 
 // Pack two floats into a 16-bit pair (element 0 in the low half), RNE.
