@@ -68,23 +68,25 @@ struct Geo {
   static constexpr int kBoxRow = kRowBytes > 128 ? 128 : kRowBytes;
   static constexpr int kBoxes = kRowBytes / kBoxRow;  // TMA boxes per tile
   static constexpr int kBoxBytes = kBoxRow * kBS;
-  static constexpr int kTileBytes = kRowBytes * kBS;
-  static constexpr int kStageBytes = 2 * kTileBytes;  // K tile + V tile
+  static constexpr int kTileBytes = kRowBytes * kBS;  // one block of K (or V)
   static constexpr int kKSteps = D / 16;              // MMA k-steps / m-tiles
+  // a ring stage holds the K and V tiles of kBPS consecutive blocks, 8 KB
+  static constexpr int kBPS = kTileBytes >= 4096 ? 1 : 4096 / kTileBytes;
+  static constexpr int kStageBytes = 2 * kBPS * kTileBytes;
   static_assert(kBoxBytes % 512 == 0, "swizzle atom alignment");
+  static_assert(kStageBytes == 8192, "8 KB stages");
 };
 
-// Shared-memory plan of one kernel instance: a 64 KB ring (8 stages of
-// 8 KB for bf16 d128, 16 stages otherwise) and, for the split path, a merge
-// buffer for two warps' per-lane records; 3 CTAs fit per SM either way.
-// Every stage is used by one consumer warp only (stages % warps == 0), so a
-// warp never waits on a stage whose previous use belongs to another warp —
-// an mbarrier parity wait cannot tell a phase from the one two ahead.
+// Shared-memory plan of one kernel instance: a 64 KB ring of 8 stages (two
+// per consumer warp) and, for the split path, a merge buffer for two warps'
+// per-lane records; 3 CTAs fit per SM either way. Every stage is used by
+// one consumer warp only (stages % warps == 0), so a warp never waits on a
+// stage whose previous use belongs to another warp — an mbarrier parity
+// wait cannot tell a phase from the one two ahead.
 template <int D, bool FP8, int NT, bool CHUNKED>
 struct Plan {
   using G = Geo<D, FP8>;
-  static constexpr int kStagesRaw = 65536 / G::kStageBytes;
-  static constexpr int kStages = kStagesRaw > 16 ? 16 : kStagesRaw;
+  static constexpr int kStages = 8;
   static constexpr int kRingBytes = kStages * G::kStageBytes;
   // per-lane merge record: acc[NT][KS] as float4, then (m0, m1, l0, l1)[NT]
   static constexpr int kLaneFloats = NT * G::kKSteps * 4 + NT * 4;
@@ -93,7 +95,6 @@ struct Plan {
   static constexpr int kBarOffset = CHUNKED ? kRingBytes + kMergeBytes : kRingBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 16 * kStages + 16;
   static_assert(kStages % kConsumerWarps == 0, "each stage belongs to one consumer warp");
-  static_assert(kStages >= 2 * kConsumerWarps, "two stages per consumer warp");
   static_assert(CHUNKED || kMergeBytes <= kRingBytes, "merge buffer fits the idle ring");
 };
 
@@ -175,69 +176,92 @@ struct WarpState {
   }
 };
 
-// One 16-token block for one consumer warp. TAIL: the block holds the end of
-// the context (`valid` < 16 tokens are real).
-template <int D, bool FP8, int NT, bool TAIL>
-__device__ __forceinline__ void attend_block(uint32_t kt, uint32_t vt, int valid, int lane,
-                                             const uint32_t (&qf)[NT][D / 16][2],
-                                             const float (&cs)[NT][2],
-                                             WarpState<D, NT> &ws) {
+// One ring stage — NB consecutive 16-token blocks — for one consumer warp,
+// as one step of the online softmax over 16 * NB tokens: the blocks' score
+// chains run interleaved and share one max/rescale. TAIL: only the first
+// `valid` (< 16 * NB) tokens of the stage are real; the rest (the end of a
+// sequence's last block, or blocks past the CTA's range, loaded as zeros)
+// are masked.
+template <int D, bool FP8, int NT, int NB, bool TAIL>
+__device__ __forceinline__ void attend_blocks(const uint32_t (&kt)[NB], const uint32_t (&vt)[NB],
+                                              int valid, int lane,
+                                              const uint32_t (&qf)[NT][D / 16][2],
+                                              const float (&cs)[NT][2], WarpState<D, NT> &ws) {
   constexpr int KS = D / 16;
   const int mi = lane >> 3;    // ldmatrix: lane supplies a row of matrix mi
   const int mrow = lane & 7;
   const int gq = lane >> 2;    // MMA group id: token row / head column
   const int qd = lane & 3;     // thread in group
 
-  // ---- scores S^T = K . Q^T  (two accumulator chains for ILP)
-  float sc[NT][2][4];
+  // ---- scores S^T = K . Q^T  (two accumulator chains per block)
+  float sc[NB][NT][2][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int b = 0; b < NB; ++b)
 #pragma unroll
-    for (int c = 0; c < 2; ++c) sc[nt][c][0] = sc[nt][c][1] = sc[nt][c][2] = sc[nt][c][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        sc[b][nt][c][0] = sc[b][nt][c][1] = sc[b][nt][c][2] = sc[b][nt][c][3] = 0.f;
   if constexpr (!FP8) {
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * ks + (mi >> 1) * 16), a0, a1, a2, a3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        mma_16816<false>(sc[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+      for (int b = 0; b < NB; ++b) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kt[b] + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * ks + (mi >> 1) * 16), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816<false>(sc[b][nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+      }
     }
   } else {
 #pragma unroll
     for (int kk = 0; kk < KS / 2; ++kk) {
-      // r0/r1: rows 0-7 / 8-15, dims [32kk, 32kk+16); r2/r3: the next 16 dims.
-      // Each register holds dims 4qd..4qd+3 of its row.
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4(kt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * kk + (mi >> 1) * 16), r0, r1, r2, r3);
-      uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-      e4m3x4_to_f16x2x2(r0, a0, a2);
-      e4m3x4_to_f16x2x2(r1, a1, a3);
-      e4m3x4_to_f16x2x2(r2, c0, c2);
-      e4m3x4_to_f16x2x2(r3, c1, c3);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816<true>(sc[nt][0], a0, a1, a2, a3, qf[nt][2 * kk][0], qf[nt][2 * kk][1]);
-        mma_16816<true>(sc[nt][1], c0, c1, c2, c3, qf[nt][2 * kk + 1][0], qf[nt][2 * kk + 1][1]);
+      for (int b = 0; b < NB; ++b) {
+        // r0/r1: rows 0-7 / 8-15, dims [32kk, 32kk+16); r2/r3: the next 16
+        // dims. Each register holds dims 4qd..4qd+3 of its row.
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(kt[b] + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * kk + (mi >> 1) * 16), r0, r1, r2, r3);
+        uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+        e4m3x4_to_f16x2x2(r0, a0, a2);
+        e4m3x4_to_f16x2x2(r1, a1, a3);
+        e4m3x4_to_f16x2x2(r2, c0, c2);
+        e4m3x4_to_f16x2x2(r3, c1, c3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<true>(sc[b][nt][0], a0, a1, a2, a3, qf[nt][2 * kk][0], qf[nt][2 * kk][1]);
+          mma_16816<true>(sc[b][nt][1], c0, c1, c2, c3, qf[nt][2 * kk + 1][0], qf[nt][2 * kk + 1][1]);
+        }
       }
     }
   }
 
-  // ---- online softmax per head column
-  uint32_t pb_hi[NT][2], pb_lo[NT][2];
+  // ---- online softmax per head column over the NB blocks' tokens
+  uint32_t pb_hi[NB][NT][2], pb_lo[NB][NT][2];
   float alpha[NT][2];
   bool rescale = false;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    float z0 = (sc[nt][0][0] + sc[nt][1][0]) * cs[nt][0];  // token gq,   head 2qd
-    float z1 = (sc[nt][0][1] + sc[nt][1][1]) * cs[nt][1];  // token gq,   head 2qd+1
-    float z2 = (sc[nt][0][2] + sc[nt][1][2]) * cs[nt][0];  // token gq+8, head 2qd
-    float z3 = (sc[nt][0][3] + sc[nt][1][3]) * cs[nt][1];  // token gq+8, head 2qd+1
+    float z[NB][4];  // token gq / gq+8 of block b, head column 2qd / 2qd+1
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) z[b][e] = (sc[b][nt][0][e] + sc[b][nt][1][e]) * cs[nt][e & 1];
     if constexpr (TAIL) {
-      if (gq >= valid) z0 = z1 = -INFINITY;
-      if (gq + 8 >= valid) z2 = z3 = -INFINITY;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int vb = valid - kBS * b;
+        if (gq >= vb) z[b][0] = z[b][1] = -INFINITY;
+        if (gq + 8 >= vb) z[b][2] = z[b][3] = -INFINITY;
+      }
     }
-    float mx0 = fmaxf(z0, z2), mx1 = fmaxf(z1, z3);
+    float mx0 = fmaxf(z[0][0], z[0][2]), mx1 = fmaxf(z[0][1], z[0][3]);
+#pragma unroll
+    for (int b = 1; b < NB; ++b) {
+      mx0 = fmaxf(mx0, fmaxf(z[b][0], z[b][2]));
+      mx1 = fmaxf(mx1, fmaxf(z[b][1], z[b][3]));
+    }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
@@ -250,22 +274,28 @@ __device__ __forceinline__ void attend_block(uint32_t kt, uint32_t vt, int valid
     rescale |= (ws.m[nt][0] != mn0) || (ws.m[nt][1] != mn1);
     ws.m[nt][0] = mn0;
     ws.m[nt][1] = mn1;
-    const float p0 = exp2f(z0 - mn0), p1 = exp2f(z1 - mn1);
-    const float p2 = exp2f(z2 - mn0), p3 = exp2f(z3 - mn1);
-    ws.l[nt][0] = ws.l[nt][0] * alpha[nt][0] + (p0 + p2);
-    ws.l[nt][1] = ws.l[nt][1] * alpha[nt][1] + (p1 + p3);
-    // P as the B operand (rows = tokens, cols = heads): build the two 8x8
-    // tiles (tokens 0-7 / 8-15) x heads in accumulator layout, transpose each
-    const uint32_t h01 = pack2<FP8>(p0, p1), h23 = pack2<FP8>(p2, p3);
-    pb_hi[nt][0] = movmatrix_trans(h01);
-    pb_hi[nt][1] = movmatrix_trans(h23);
-    if constexpr (!FP8) {
-      float u0, u1, u2, u3;
-      unpack2<false>(h01, u0, u1);
-      unpack2<false>(h23, u2, u3);
-      pb_lo[nt][0] = movmatrix_trans(pack2<false>(p0 - u0, p1 - u1));
-      pb_lo[nt][1] = movmatrix_trans(pack2<false>(p2 - u2, p3 - u3));
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const float p0 = exp2f(z[b][0] - mn0), p1 = exp2f(z[b][1] - mn1);
+      const float p2 = exp2f(z[b][2] - mn0), p3 = exp2f(z[b][3] - mn1);
+      s0 += p0 + p2;
+      s1 += p1 + p3;
+      // P as the B operand (rows = tokens, cols = heads): build the two 8x8
+      // tiles (tokens 0-7 / 8-15) x heads in accumulator layout, transpose
+      const uint32_t h01 = pack2<FP8>(p0, p1), h23 = pack2<FP8>(p2, p3);
+      pb_hi[b][nt][0] = movmatrix_trans(h01);
+      pb_hi[b][nt][1] = movmatrix_trans(h23);
+      if constexpr (!FP8) {
+        float u0, u1, u2, u3;
+        unpack2<false>(h01, u0, u1);
+        unpack2<false>(h23, u2, u3);
+        pb_lo[b][nt][0] = movmatrix_trans(pack2<false>(p0 - u0, p1 - u1));
+        pb_lo[b][nt][1] = movmatrix_trans(pack2<false>(p2 - u2, p3 - u3));
+      }
     }
+    ws.l[nt][0] = ws.l[nt][0] * alpha[nt][0] + s0;
+    ws.l[nt][1] = ws.l[nt][1] * alpha[nt][1] + s1;
   }
   if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -279,56 +309,67 @@ __device__ __forceinline__ void attend_block(uint32_t kt, uint32_t vt, int valid
       }
   }
 
-  // ---- O^T += V^T . P ; V of tokens >= valid is zeroed (tail block only)
-  uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-  if constexpr (TAIL) {
-    mlo = (2 * qd < valid ? 0x0000ffffu : 0u) | (2 * qd + 1 < valid ? 0xffff0000u : 0u);
-    mhi = (2 * qd + 8 < valid ? 0x0000ffffu : 0u) | (2 * qd + 9 < valid ? 0xffff0000u : 0u);
+  // ---- O^T += V^T . P ; V of masked tokens is zeroed (tail stage only):
+  // these fragments hold tokens (2qd, 2qd+1) and (2qd+8, 2qd+9)
+  uint32_t mlo[NB], mhi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const int vb = valid - kBS * b;
+    mlo[b] = (2 * qd < vb ? 0x0000ffffu : 0u) | (2 * qd + 1 < vb ? 0xffff0000u : 0u);
+    mhi[b] = (2 * qd + 8 < vb ? 0x0000ffffu : 0u) | (2 * qd + 9 < vb ? 0xffff0000u : 0u);
   }
   if constexpr (!FP8) {
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4_trans(vt + swz<D, FP8>((mi >> 1) * 8 + mrow, 32 * mt + (mi & 1) * 16), a0, a1, a2, a3);
-      if constexpr (TAIL) {
-        a0 &= mlo;
-        a1 &= mlo;
-        a2 &= mhi;
-        a3 &= mhi;
-      }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
-        mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_lo[nt][0], pb_lo[nt][1]);
+      for (int b = 0; b < NB; ++b) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(vt[b] + swz<D, FP8>((mi >> 1) * 8 + mrow, 32 * mt + (mi & 1) * 16), a0, a1,
+                      a2, a3);
+        if constexpr (TAIL) {
+          a0 &= mlo[b];
+          a1 &= mlo[b];
+          a2 &= mhi[b];
+          a3 &= mhi[b];
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_hi[b][nt][0], pb_hi[b][nt][1]);
+          mma_16816<false>(ws.acc[nt][mt], a0, a1, a2, a3, pb_lo[b][nt][0], pb_lo[b][nt][1]);
+        }
       }
     }
   } else {
 #pragma unroll
     for (int cc = 0; cc < KS / 2; ++cc) {
-      // r0/r1: tokens 0-7 / 8-15 of dims [32cc, 32cc+16); r2/r3: next 16
-      // dims. Bytes of r: (t,2g) (t,2g+1) (t+1,2g) (t+1,2g+1) with
-      // t = 2qd, g = gq; regroup into token pairs per dim, then widen.
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4_trans(vt + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * cc + (mi >> 1) * 16), r0, r1, r2, r3);
-      uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-      e4m3x4_to_f16x2x2(prmt(r0, 0x3120), a0, a1);
-      e4m3x4_to_f16x2x2(prmt(r1, 0x3120), a2, a3);
-      e4m3x4_to_f16x2x2(prmt(r2, 0x3120), c0, c1);
-      e4m3x4_to_f16x2x2(prmt(r3, 0x3120), c2, c3);
-      if constexpr (TAIL) {
-        a0 &= mlo;
-        a1 &= mlo;
-        a2 &= mhi;
-        a3 &= mhi;
-        c0 &= mlo;
-        c1 &= mlo;
-        c2 &= mhi;
-        c3 &= mhi;
-      }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816<true>(ws.acc[nt][2 * cc], a0, a1, a2, a3, pb_hi[nt][0], pb_hi[nt][1]);
-        mma_16816<true>(ws.acc[nt][2 * cc + 1], c0, c1, c2, c3, pb_hi[nt][0], pb_hi[nt][1]);
+      for (int b = 0; b < NB; ++b) {
+        // r0/r1: tokens 0-7 / 8-15 of dims [32cc, 32cc+16); r2/r3: next 16
+        // dims. Bytes of r: (t,2g) (t,2g+1) (t+1,2g) (t+1,2g+1) with
+        // t = 2qd, g = gq; regroup into token pairs per dim, then widen.
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_trans(vt[b] + swz<D, FP8>((mi & 1) * 8 + mrow, 32 * cc + (mi >> 1) * 16), r0, r1,
+                      r2, r3);
+        uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+        e4m3x4_to_f16x2x2(prmt(r0, 0x3120), a0, a1);
+        e4m3x4_to_f16x2x2(prmt(r1, 0x3120), a2, a3);
+        e4m3x4_to_f16x2x2(prmt(r2, 0x3120), c0, c1);
+        e4m3x4_to_f16x2x2(prmt(r3, 0x3120), c2, c3);
+        if constexpr (TAIL) {
+          a0 &= mlo[b];
+          a1 &= mlo[b];
+          a2 &= mhi[b];
+          a3 &= mhi[b];
+          c0 &= mlo[b];
+          c1 &= mlo[b];
+          c2 &= mhi[b];
+          c3 &= mhi[b];
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816<true>(ws.acc[nt][2 * cc], a0, a1, a2, a3, pb_hi[b][nt][0], pb_hi[b][nt][1]);
+          mma_16816<true>(ws.acc[nt][2 * cc + 1], c0, c1, c2, c3, pb_hi[b][nt][0], pb_hi[b][nt][1]);
+        }
       }
     }
   }
@@ -454,6 +495,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   using PL = Plan<D, FP8, NT, CHUNKED>;
   constexpr int NS = PL::kStages;
   constexpr int KS = G::kKSteps;
+  constexpr int BPS = G::kBPS;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -486,6 +528,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
   if (bad_len && threadIdx.x == 0 && chunk == 0) raise_error(kErrContextClamp);
   const int nblk = j1 - j0;
+  const int nst = (nblk + BPS - 1) / BPS;  // ring stages this CTA streams
+  const int tok_end = min(L, j1 * kBS);    // tokens past this are masked
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -508,41 +552,50 @@ __global__ void __launch_bounds__(kDecodeThreads)
     int issued = 0;
     bool ok = true;
     bool bad_id = false;
-    for (int jb = 0; jb < nblk && ok; jb += 32) {
-      const int mine = (jb + lane < nblk) ? bt[j0 + jb + lane] : 0;
-      const int cnt = min(32, nblk - jb);
-      for (int i = 0; i < cnt; ++i) {
-        const int phys = __shfl_sync(0xffffffffu, mine, i);
+    // 32 table entries per coalesced load; a stage never straddles two
+    // windows because BPS divides 32
+    for (int jb = 0; jb < nst * BPS && ok; jb += 32) {
+      const int mine = (jb + lane < nblk) ? bt[j0 + jb + lane] : -1;
+      const int i_end = min(nst, (jb + 32) / BPS);
+      for (int i = jb / BPS; i < i_end; ++i) {
+        int phys[BPS];
+#pragma unroll
+        for (int b = 0; b < BPS; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, i * BPS + b - jb);
         if (lane == 0) {
-          const int it = jb + i;
-          const int st = it % NS;
-          if (it >= NS) {
+          const int st = i % NS;
+          if (i >= NS && !mbar_try_wait(empty0 + 8u * st, ((i / NS) - 1) & 1)) {
             if (*s_abort) {
               ok = false;
-            } else if (!mbar_wait_bounded(empty0 + 8u * st, ((it / NS) - 1) & 1, kWaitLimitNs)) {
+            } else if (!mbar_wait_bounded(empty0 + 8u * st, ((i / NS) - 1) & 1, kWaitLimitNs)) {
               ok = false;
               *s_abort = 1;
               raise_error(kErrWaitTimeout);
             }
           }
           if (ok) {
-            int y;
-            if (phys < 0 || phys >= p.num_blocks) {
-              y = total_rows;  // whole box out of range: TMA fills zeros
-              bad_id = true;
-            } else {
-              y = (phys * p.num_kv_heads + h) * kBS;
-            }
             const uint32_t fb = full0 + 8u * st;
             const uint32_t kdst = ring + st * G::kStageBytes;
-            const uint32_t vdst = kdst + G::kTileBytes;
+            const uint32_t vdst = kdst + BPS * G::kTileBytes;
             mbar_arrive_expect_tx(fb, G::kStageBytes);
 #pragma unroll
-            for (int b = 0; b < G::kBoxes; ++b) {
-              tma_load_2d(kdst + b * G::kBoxBytes, &tmap_k, fb, b * (G::kBoxRow / G::kEB), y);
-              tma_load_2d(vdst + b * G::kBoxBytes, &tmap_v, fb, b * (G::kBoxRow / G::kEB), y);
+            for (int b = 0; b < BPS; ++b) {
+              const bool real = i * BPS + b < nblk;
+              int y;
+              if (!real || phys[b] < 0 || phys[b] >= p.num_blocks) {
+                y = total_rows;  // whole box out of range: TMA fills zeros
+                bad_id |= real;
+              } else {
+                y = (phys[b] * p.num_kv_heads + h) * kBS;
+              }
+#pragma unroll
+              for (int x = 0; x < G::kBoxes; ++x) {
+                tma_load_2d(kdst + b * G::kTileBytes + x * G::kBoxBytes, &tmap_k, fb,
+                            x * (G::kBoxRow / G::kEB), y);
+                tma_load_2d(vdst + b * G::kTileBytes + x * G::kBoxBytes, &tmap_v, fb,
+                            x * (G::kBoxRow / G::kEB), y);
+              }
             }
-            issued = it + 1;
+            issued = i + 1;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -553,8 +606,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
       if (bad_id) raise_error(kErrBlockRange);
       // No bulk copy may still be landing in this CTA's shared memory when
       // it moves on: wait (bounded) for the last load of every stage.
-      for (int it = max(0, issued - NS); it < issued; ++it)
-        mbar_wait_bounded(full0 + 8u * (it % NS), (it / NS) & 1, kWaitLimitNs);
+      for (int i = max(0, issued - NS); i < issued; ++i)
+        mbar_wait_bounded(full0 + 8u * (i % NS), (i / NS) & 1, kWaitLimitNs);
     }
     if (!CHUNKED) __syncthreads();  // single-pass: the merge reuses the ring
     return;
@@ -619,35 +672,40 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
   }
 
-  // Blocks of this warp: it = warp, warp + 4, ... over [0, nblk). Split
-  // ranges are whole partitions of pb blocks, pb a multiple of 4, so every
-  // warp crosses a partition boundary at the same iteration.
+  // Stages of this warp: i = warp, warp + 4, ... over [0, nst). In a split
+  // chunk every partition is a whole number of rounds (pb / BPS stages, a
+  // multiple of 4), so all warps cross a partition boundary together.
+  const int spb = CHUNKED ? pb / BPS : 0;
   bool aborted = false;
-  int it = warp;
+  int i = warp;
   for (int pi = 0; pi < npart; ++pi) {
-    const int it_end = CHUNKED ? min(nblk, (pi + 1) * pb) : nblk;
-    for (; it < it_end; it += kConsumerWarps) {
-      if (!aborted) {
-        const int st = it % NS;
-        const bool got = mbar_wait_bounded(full0 + 8u * st, (it / NS) & 1, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, got)) {
-          aborted = true;
-          if (lane == 0) {
-            *s_abort = 1;
-            raise_error(kErrWaitTimeout);
-          }
-          continue;
+    const int i_end = (CHUNKED && npart > 1) ? min(nst, (pi + 1) * spb) : nst;
+    for (; i < i_end; i += kConsumerWarps) {
+      if (aborted) continue;
+      const int st = i % NS;
+      const bool got = mbar_wait_bounded(full0 + 8u * st, (i / NS) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        aborted = true;
+        if (lane == 0) {
+          *s_abort = 1;
+          raise_error(kErrWaitTimeout);
         }
-        const uint32_t kt = ring + st * G::kStageBytes;
-        const uint32_t vt = kt + G::kTileBytes;
-        const int valid = L - (j0 + it) * kBS;
-        if (valid >= kBS)
-          attend_block<D, FP8, NT, false>(kt, vt, kBS, lane, qf, cs, ws);
-        else
-          attend_block<D, FP8, NT, true>(kt, vt, valid, lane, qf, cs, ws);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8u * st);
+        continue;
       }
+      const uint32_t k0 = ring + st * G::kStageBytes;
+      uint32_t kt[BPS], vt[BPS];
+#pragma unroll
+      for (int b = 0; b < BPS; ++b) {
+        kt[b] = k0 + b * G::kTileBytes;
+        vt[b] = k0 + (BPS + b) * G::kTileBytes;
+      }
+      const int valid = tok_end - (j0 + i * BPS) * kBS;  // real tokens in this stage
+      if (valid >= BPS * kBS)
+        attend_blocks<D, FP8, NT, BPS, false>(kt, vt, BPS * kBS, lane, qf, cs, ws);
+      else
+        attend_blocks<D, FP8, NT, BPS, true>(kt, vt, valid, lane, qf, cs, ws);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8u * st);
     }
     if (CHUNKED) {
       consumer_bar_sync();  // the previous partition's merge has read mbuf
@@ -660,7 +718,6 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
   }
 }
-
 
 // Combine the partitions of one (sequence, query head):
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.

@@ -126,13 +126,13 @@ pa_status dispatch_nt(int nt, bool chunked, const void *kc, const void *vc, int 
 }
 
 // Consecutive partitions per CTA in the split path: about 1 MB of K/V per
-// CTA, while keeping at least four CTAs per SM in the grid. Chunks need
-// partitions of a multiple of 4 blocks (one per consumer warp per round).
-int partitions_per_cta(int64_t units, int64_t P, int psize, int num_kv_heads_unused,
-                       int head_dim, int eb, int sms) {
-  (void)num_kv_heads_unused;
+// CTA, while keeping at least four CTAs per SM in the grid. Chunks of more
+// than one partition need partitions of a whole number of ring rounds
+// (4 consumer warps x `bps` blocks per stage).
+int partitions_per_cta(int64_t units, int64_t P, int psize, int head_dim, int eb, int bps,
+                       int sms) {
   const int pb = psize / pa::kBS;
-  if (pb % pa::kConsumerWarps != 0) return 1;
+  if (pb % (pa::kConsumerWarps * bps) != 0) return 1;
   const int64_t part_bytes = static_cast<int64_t>(psize) * head_dim * eb * 2;
   int64_t ppc = std::max<int64_t>(1, (int64_t{1} << 20) / std::max<int64_t>(part_bytes, 1));
   ppc = std::min<int64_t>(ppc, P);
@@ -274,10 +274,10 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
     p.ws_l = reinterpret_cast<float *>(ws + o_bytes + m_bytes);
     p.partition_blocks = psize / pa::kBS;
     p.max_partitions = static_cast<int>(P);
+    const int eb = kv_dtype == PA_KV_BF16 ? 2 : 1;
+    const int bps = (pa::kBS * head_dim * eb) >= 4096 ? 1 : 4096 / (pa::kBS * head_dim * eb);
     p.partitions_per_cta = partitions_per_cta(static_cast<int64_t>(num_seqs) * num_kv_heads, P,
-                                              psize, num_kv_heads, head_dim,
-                                              kv_dtype == PA_KV_BF16 ? 2 : 1,
-                                              device_sm_count(dev));
+                                              psize, head_dim, eb, bps, device_sm_count(dev));
     grid_x = static_cast<int>((P + p.partitions_per_cta - 1) / p.partitions_per_cta);
   }
 
