@@ -316,7 +316,7 @@ def _auto_split(batch, ws) -> bool:
     sms = torch.cuda.get_device_properties(batch.device).multi_processor_count
     units = w.num_seqs * w.num_kv_heads
     cap = min(batch.max_context_len, batch.max_blocks * 16)
-    return (units < 6 * sms or cap > 4096) and cap > 512
+    return (units < 2 * 3 * sms or cap > 16384) and cap > 512
 
 
 def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):

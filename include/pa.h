@@ -214,6 +214,29 @@ PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache,
                          const int64_t *block_pairs, int num_pairs,
                          size_t block_bytes, int num_blocks, void *stream);
 
+/* Swap blocks between two caches of the same block geometry — typically the
+ * GPU cache and a cache in page-locked host memory — for preemption: a
+ * request's KV blocks are moved to CPU memory and back later ([Day28] §六
+ * question 4, §七 and FAQ Q3: watermark, preemption, swapping). For each
+ * pair (src, dst): dst cache block dst <- src cache block src, K and V
+ * alike. One kernel launch moves every pair; host memory is read or written
+ * through its device mapping, so the copy runs at the host link's speed.
+ *   dst_*, src_*  caches [num_blocks][Hkv][16][D]: device memory of the
+ *                 current device, managed memory, or page-locked host memory
+ *                 registered with CUDA (cudaHostAlloc, cudaHostRegister).
+ *                 Pageable host memory returns PA_ERR_INVALID_ARG (nothing
+ *                 launched). 16-byte aligned.
+ *   block_pairs   int64 [num_pairs][2] (src, dst), in device or page-locked
+ *                 host memory. A pair outside its cache is skipped and flagged
+ *                 PA_DEVERR_PAIR_RANGE. Destinations must be distinct.
+ *   block_bytes   bytes of one block of ONE cache, multiple of 16. */
+PA_API pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache,
+                                const void *src_k_cache,
+                                const void *src_v_cache,
+                                const int64_t *block_pairs, int num_pairs,
+                                size_t block_bytes, int src_num_blocks,
+                                int dst_num_blocks, void *stream);
+
 /* Synchronise the current device, then read and clear its device error word
  * (a bitwise OR of PA_DEVERR_* since the last read) into *code_out (host).
  * Returns PA_ERR_DEVICE when the word was non-zero, PA_OK when it was zero,
@@ -271,7 +294,52 @@ PA_API pa_status pa_pool_block_tables(const pa_pool *pool, const int64_t *seq_id
                                int n, int32_t *tables_out,
                                int max_blocks_per_seq, int32_t *ctx_out);
 
-PA_API int pa_pool_num_free(const pa_pool *pool);          /* -1 if pool is NULL   */
+/* Automatic prefix caching ([Ch7] §7.1 前缀共享 and §"vLLM 关键参数速记"
+ * --enable-prefix-caching; [Day28] §4.2: CoW sharing makes prefix caching a
+ * natural consequence of paging, §七: shared system prompts skip prefill).
+ * With caching enabled, every block that becomes full through
+ * pa_pool_append_tokens gets a content key: its parent block's key and its
+ * 16 token ids. A later append whose next whole block of tokens matches a
+ * cached block (compared id by id, so a key collision can never alias) takes
+ * that block (refcount + 1) instead of a new one — up to the first miss —
+ * and its slots are returned as -1: that KV is already in the cache and
+ * pa_reshape_and_cache skips negative slots. A block whose last user leaves
+ * keeps its key and stays findable until a fresh block is needed, when the
+ * least recently freed such block is reused. Disabling forgets all keys. */
+PA_API pa_status pa_pool_enable_prefix_caching(pa_pool *pool, int enable);
+
+/* pa_pool_append with the new tokens' ids (int32 [n_tokens], host):
+ * *n_cached_out receives how many leading tokens were found in the cache
+ * (a multiple of 16; their slots are -1). Plain pa_pool_append on a
+ * sequence ends its keyed prefix (later blocks get no key). */
+PA_API pa_status pa_pool_append_tokens(pa_pool *pool, int64_t seq_id,
+                                       const int32_t *token_ids, int n_tokens,
+                                       int64_t *slots_out,
+                                       int64_t *cow_pairs_out, int *n_cow_out,
+                                       int *n_cached_out);
+
+/* Number of blocks currently findable by content (in use or evictable). */
+PA_API int pa_pool_num_cached(const pa_pool *pool);
+
+/* Preemption by swapping ([Day28] §六 question 4, §七, FAQ Q3): move a
+ * sequence from the GPU pool to a CPU pool (swap_out) or back (swap_in).
+ * Every block of the sequence gets a block in the destination pool; the
+ * (source block, destination block) pairs are written to pairs_out
+ * [n][2] (at most max_pairs), *n_pairs_out = n, for pa_swap_blocks to move
+ * the data. Source references are dropped (a block still shared by another
+ * sequence stays where it is); the moved sequence owns private copies.
+ * PA_ERR_OUT_OF_BLOCKS (destination too full) and PA_ERR_INVALID_ARG
+ * (max_pairs too small, id already in the destination) change nothing. */
+PA_API pa_status pa_pool_swap_out(pa_pool *gpu_pool, pa_pool *cpu_pool,
+                                  int64_t seq_id, int64_t *pairs_out,
+                                  int max_pairs, int *n_pairs_out);
+PA_API pa_status pa_pool_swap_in(pa_pool *gpu_pool, pa_pool *cpu_pool,
+                                 int64_t seq_id, int64_t *pairs_out,
+                                 int max_pairs, int *n_pairs_out);
+
+/* Blocks that can be handed out: free ones plus cached ones no sequence
+ * uses (-1 if pool is NULL). */
+PA_API int pa_pool_num_free(const pa_pool *pool);
 PA_API int pa_pool_refcount(const pa_pool *pool, int block_id); /* -1 if invalid   */
 /* Length (tokens) and block count of a sequence; -1 if unknown. */
 PA_API int64_t pa_pool_seq_len(const pa_pool *pool, int64_t seq_id);

@@ -75,6 +75,8 @@ def _load():
     lib.oracle_reshape_and_cache.restype = i32
     lib.oracle_copy_blocks.argtypes = [vp, vp, vp, i32, i64, i32]
     lib.oracle_copy_blocks.restype = i32
+    lib.oracle_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32]
+    lib.oracle_swap_blocks.restype = i32
     lib.oracle_paged_decode.argtypes = [vp, vp, vp, vp, i32, f64, f64, vp, i32,
                                         vp, i32, i32, i32, i32, i32, i32, f64,
                                         vp, i32]
@@ -172,6 +174,17 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray,
     _check(_load().oracle_copy_blocks(_ptr(k_cache), _ptr(v_cache),
                                       _ptr(pairs), pairs.shape[0],
                                       block_bytes, NB), "copy_blocks")
+
+
+def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k: np.ndarray,
+                src_v: np.ndarray, pairs: np.ndarray) -> None:
+    """dst[dst_id] = src[src_id] for each (src_id, dst_id) pair, K and V."""
+    pairs = np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2)
+    assert dst_k[0].nbytes == src_k[0].nbytes
+    _check(_load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k),
+                                      _ptr(src_v), _ptr(pairs), pairs.shape[0],
+                                      src_k[0].nbytes, src_k.shape[0],
+                                      dst_k.shape[0]), "swap_blocks")
 
 
 # ---------------------------------------------------------------- decode

@@ -202,6 +202,26 @@ int oracle_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs,
   return 0;
 }
 
+/* Swap: copy physical blocks between two caches (GPU pool <-> host pool),
+ * dst_cache[dst] = src_cache[src] for each (src, dst) pair, K and V alike.
+ * Preemption moves a request's KV blocks to CPU memory and back ([Day28]
+ * §六 question 4, §七 and FAQ Q3: watermark, preemption, swapping). */
+int oracle_swap_blocks(void *dst_k, void *dst_v, const void *src_k,
+                       const void *src_v, const int64_t *pairs, int num_pairs,
+                       int64_t block_bytes, int src_num_blocks,
+                       int dst_num_blocks) {
+  int i;
+  for (i = 0; i < num_pairs; ++i) {
+    int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return 1;
+    memcpy((char *)dst_k + dst * block_bytes,
+           (const char *)src_k + src * block_bytes, (size_t)block_bytes);
+    memcpy((char *)dst_v + dst * block_bytes,
+           (const char *)src_v + src * block_bytes, (size_t)block_bytes);
+  }
+  return 0;
+}
+
 /* --------------------------------------------------------------- attention */
 
 static double cache_value(const void *cache, int kv_dtype, double scale,

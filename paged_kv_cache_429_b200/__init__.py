@@ -7,8 +7,10 @@ functions carry the names of the C entry points (include/pa.h):
     pa_decode               decode-step attention through block tables
     pa_reshape_and_cache    scatter new K/V into cache slots (bf16 / fp8)
     pa_copy_blocks          copy-on-write block copies
+    pa_swap_blocks          block copies between the GPU cache and pinned host memory
+    pa_decode_no_alloc      split-context decode with the library's fixed scratch
     pa_decode_workspace_size, pa_get_device_error, pa_status_string
-    BlockPool               host block pool (pa_pool_*)
+    BlockPool               host block pool (pa_pool_*), incl. swap_out / swap_in
 
 Cache layout: [num_blocks][num_kv_heads][16][head_dim], bf16 or
 float8_e4m3fn (uint8 is accepted for fp8 bytes).
@@ -27,7 +29,8 @@ from ._lib import STATUS_NAMES, LibraryNotBuilt
 __all__ = [
     "PA_KV_BF16", "PA_KV_FP8_E4M3", "BLOCK_SIZE", "PagedAttentionError",
     "LibraryNotBuilt", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
-    "pa_decode_workspace_size", "pa_get_device_error", "pa_status_string",
+    "pa_swap_blocks", "pa_decode_workspace_size", "pa_get_device_error",
+    "pa_status_string",
     "BlockPool", "kv_dtype_of",
 ]
 
@@ -162,6 +165,29 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor,
     _ok(rc, "pa_copy_blocks")
 
 
+def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                   src_v: torch.Tensor, block_pairs: torch.Tensor, *,
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """dst[dst_id] = src[src_id] for each (src_id, dst_id) pair of
+    block_pairs (int64 [n][2]); each cache is on the current CUDA device or
+    in pinned host memory (torch ``pin_memory()``)."""
+    for name, t in (("dst_k", dst_k), ("dst_v", dst_v), ("src_k", src_k), ("src_v", src_v)):
+        _need(t, name, (torch.bfloat16, torch.float8_e4m3fn, torch.uint8), 4, cuda=False)
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be on the GPU or in pinned host memory")
+    _need(block_pairs, "block_pairs", (torch.int64,), 2, cuda=False)
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype:
+        raise ValueError("source and destination caches differ in block geometry")
+    n = block_pairs.shape[0]
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    dev = dst_k.device if dst_k.is_cuda else (src_k.device if src_k.is_cuda else None)
+    rc = _lib.lib().pa_swap_blocks(
+        dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(),
+        block_pairs.data_ptr() if n else None, n, block_bytes, src_k.shape[0],
+        dst_k.shape[0], _stream_ptr(stream, dev))
+    _ok(rc, "pa_swap_blocks")
+
+
 def pa_get_device_error() -> int:
     """Synchronise the current device; return and clear its error bits."""
     code = ctypes.c_uint32(0)
@@ -209,6 +235,28 @@ class BlockPool:
             "pa_pool_append")
         return slots, ((int(pair[0]), int(pair[1])) if ncow.value else None)
 
+    def enable_prefix_caching(self, enable: bool = True) -> None:
+        _ok(self._lib.pa_pool_enable_prefix_caching(self._h, int(enable)),
+            "pa_pool_enable_prefix_caching")
+
+    def append_tokens(self, seq_id: int, token_ids):
+        """Append tokens with their ids (prefix caching). Returns (slots,
+        cow pair or None, n_cached): slots of cached tokens are -1."""
+        ids = np.ascontiguousarray(token_ids, dtype=np.int32)
+        n = ids.size
+        slots = np.empty(max(n, 0), dtype=np.int64)
+        pair = np.zeros(2, dtype=np.int64)
+        ncow, ncached = ctypes.c_int(0), ctypes.c_int(0)
+        _ok(self._lib.pa_pool_append_tokens(
+            self._h, seq_id, ids.ctypes.data if n else None, n,
+            slots.ctypes.data if n else None, pair.ctypes.data, ctypes.byref(ncow),
+            ctypes.byref(ncached)), "pa_pool_append_tokens")
+        return slots, ((int(pair[0]), int(pair[1])) if ncow.value else None), ncached.value
+
+    @property
+    def num_cached(self) -> int:
+        return int(self._lib.pa_pool_num_cached(self._h))
+
     def free_seq(self, seq_id: int) -> None:
         _ok(self._lib.pa_pool_free_seq(self._h, seq_id), "pa_pool_free_seq")
 
@@ -222,6 +270,24 @@ class BlockPool:
                                            tables.ctypes.data, max_blocks_per_seq,
                                            ctx.ctypes.data), "pa_pool_block_tables")
         return tables, ctx
+
+    def _move(self, fn: str, cpu_pool: "BlockPool", seq_id: int) -> np.ndarray:
+        n_max = max(self.seq_num_blocks(seq_id), cpu_pool.seq_num_blocks(seq_id), 1)
+        pairs = np.zeros((n_max, 2), dtype=np.int64)
+        n = ctypes.c_int(0)
+        _ok(getattr(self._lib, fn)(self._h, cpu_pool._h, seq_id, pairs.ctypes.data,
+                                   n_max, ctypes.byref(n)), fn)
+        return pairs[:n.value]
+
+    def swap_out(self, cpu_pool: "BlockPool", seq_id: int) -> np.ndarray:
+        """Move seq_id from this (GPU) pool to cpu_pool; returns the
+        (gpu block, cpu block) pairs to copy with pa_swap_blocks."""
+        return self._move("pa_pool_swap_out", cpu_pool, seq_id)
+
+    def swap_in(self, cpu_pool: "BlockPool", seq_id: int) -> np.ndarray:
+        """Move seq_id from cpu_pool back to this (GPU) pool; returns the
+        (cpu block, gpu block) pairs to copy with pa_swap_blocks."""
+        return self._move("pa_pool_swap_in", cpu_pool, seq_id)
 
     @property
     def num_free(self) -> int:

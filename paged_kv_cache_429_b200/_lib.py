@@ -32,6 +32,7 @@ SIGNATURES = {
     "pa_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                     _i32, _i32, _i32, _f32, _f32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _sz, _i32, _vp]),
+    "pa_swap_blocks": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _sz, _i32, _i32, _vp]),
     "pa_get_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint32)]),
     "pa_pool_create": (_vp, [_i32, _i32]),
     "pa_pool_destroy": (None, [_vp]),
@@ -41,6 +42,12 @@ SIGNATURES = {
     "pa_pool_append": (_i32, [_vp, _i64, _i32, _vp, _vp, ctypes.POINTER(_i32)]),
     "pa_pool_free_seq": (_i32, [_vp, _i64]),
     "pa_pool_block_tables": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp]),
+    "pa_pool_enable_prefix_caching": (_i32, [_vp, _i32]),
+    "pa_pool_append_tokens": (_i32, [_vp, _i64, _vp, _i32, _vp, _vp, ctypes.POINTER(_i32),
+                                     ctypes.POINTER(_i32)]),
+    "pa_pool_num_cached": (_i32, [_vp]),
+    "pa_pool_swap_out": (_i32, [_vp, _vp, _i64, _vp, _i32, ctypes.POINTER(_i32)]),
+    "pa_pool_swap_in": (_i32, [_vp, _vp, _i64, _vp, _i32, ctypes.POINTER(_i32)]),
     "pa_pool_num_free": (_i32, [_vp]),
     "pa_pool_refcount": (_i32, [_vp, _i32]),
     "pa_pool_seq_len": (_i64, [_vp, _i64]),

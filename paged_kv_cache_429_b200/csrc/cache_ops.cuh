@@ -8,8 +8,10 @@
 // whole rows, so reads and writes are coalesced 16-byte accesses.
 //
 // copy_blocks — copy-on-write of a shared block ("vLLM 与 PagedAttention：
-// 把 GPU 显存当操作系统内存管" §PagedAttention 写时复制; Day 28 §六 item 4).
-// Each CTA streams one (pair, cache) block with 16-byte loads/stores.
+// 把 GPU 显存当操作系统内存管" §PagedAttention 写时复制; Day 28 §六 item 4)
+// and swapping of blocks to and from host memory (Day 28 §六 question 4,
+// §七, FAQ Q3). Each CTA streams one (pair, cache) block with 16-byte
+// loads/stores, four in flight per thread.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -80,21 +82,26 @@ __global__ void __launch_bounds__(kCacheThreads)
   }
 }
 
-// grid.x = 2 * num_pairs (pair i: CTA 2i copies K, 2i+1 copies V)
+// dst[dst_id] = src[src_id] for each (src_id, dst_id) pair; grid.x =
+// 2 * num_pairs (pair i: CTA 2i copies the K block, 2i+1 the V block).
+// Serves copy-on-write (both caches the same) and swapping (one side in
+// page-locked host memory, reached through its device mapping).
 __global__ void __launch_bounds__(kCacheThreads)
-    copy_blocks_kernel(uint4 *k_cache, uint4 *v_cache,
+    copy_blocks_kernel(uint4 *dst_k, uint4 *dst_v, const uint4 *src_k, const uint4 *src_v,
                        const int64_t *__restrict__ pairs, int64_t block_chunks,
-                       int num_blocks) {
+                       int src_num_blocks, int dst_num_blocks) {
   const int pair = blockIdx.x >> 1;
-  uint4 *cache = (blockIdx.x & 1) ? v_cache : k_cache;
+  const bool is_v = blockIdx.x & 1;
+  const uint4 *src_base = is_v ? src_v : src_k;
+  uint4 *dst_base = is_v ? dst_v : dst_k;
   const int64_t src = pairs[2 * pair];
   const int64_t dst = pairs[2 * pair + 1];
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-    if (threadIdx.x == 0 && (blockIdx.x & 1) == 0) raise_error(kErrPairRange);
+  if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
+    if (threadIdx.x == 0 && !is_v) raise_error(kErrPairRange);
     return;
   }
-  const uint4 *s = cache + src * block_chunks;
-  uint4 *d = cache + dst * block_chunks;
+  const uint4 *s = src_base + src * block_chunks;
+  uint4 *d = dst_base + dst * block_chunks;
   int64_t i = threadIdx.x;
   for (; i + 3 * kCacheThreads < block_chunks; i += 4 * kCacheThreads) {
     const uint4 x0 = s[i];

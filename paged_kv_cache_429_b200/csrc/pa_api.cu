@@ -227,12 +227,15 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   // ---- path choice
   int psize = partition_size;
   if (psize < 0) {
+    // Single-pass when the (sequence, KV head) pairs fill at least two full
+    // waves of resident CTAs (3 per SM) and contexts are not long enough for
+    // the last wave's imbalance to matter; otherwise split the contexts.
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
-    const bool wide = units >= 6LL * device_sm_count(dev);
+    const bool wide = units >= 2LL * 3 * device_sm_count(dev);
     const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap,
                                             kDefaultPartition);
     const bool have_ws = workspace && aligned(workspace, 256) && workspace_bytes >= need;
-    psize = (!wide || ctx_cap > 4096) && have_ws && ctx_cap > kDefaultPartition
+    psize = (!wide || ctx_cap > 16384) && have_ws && ctx_cap > kDefaultPartition
                 ? kDefaultPartition
                 : 0;
   }
@@ -357,8 +360,64 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pair
   if (num_pairs > (1 << 30)) return PA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   pa::copy_blocks_kernel<<<2 * num_pairs, pa::kCacheThreads, 0, st>>>(
-      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_pairs,
-      static_cast<int64_t>(block_bytes / 16), num_blocks);
+      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache),
+      static_cast<const uint4 *>(k_cache), static_cast<const uint4 *>(v_cache), block_pairs,
+      static_cast<int64_t>(block_bytes / 16), num_blocks, num_blocks);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Device-accessible address of `p` on the current device: device memory of
+// this device, managed memory, or page-locked host memory registered with
+// CUDA (through its device mapping). nullptr for anything else, e.g.
+// pageable host memory, which a kernel must never be given.
+static const void *device_view(const void *p, int dev) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the (non-sticky) error the query left
+    return nullptr;
+  }
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+      return a.device == dev ? p : nullptr;
+    case cudaMemoryTypeManaged:
+      return p;
+    case cudaMemoryTypeHost: {
+      if (!a.devicePointer) return nullptr;
+      // keep the byte offset of p inside its registered range
+      return static_cast<const char *>(a.devicePointer) +
+             (static_cast<const char *>(p) - static_cast<const char *>(a.hostPointer));
+    }
+    default:
+      return nullptr;
+  }
+}
+
+pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k_cache,
+                         const void *src_v_cache, const int64_t *block_pairs, int num_pairs,
+                         size_t block_bytes, int src_num_blocks, int dst_num_blocks,
+                         void *stream) {
+  if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 || block_bytes == 0 ||
+      block_bytes % 16 != 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !block_pairs)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(dst_k_cache, 16) || !aligned(dst_v_cache, 16) || !aligned(src_k_cache, 16) ||
+      !aligned(src_v_cache, 16) || !aligned(block_pairs, 8))
+    return PA_ERR_INVALID_ARG;
+  if (num_pairs > (1 << 30)) return PA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const void *dk = device_view(dst_k_cache, dev), *dv = device_view(dst_v_cache, dev);
+  const void *sk = device_view(src_k_cache, dev), *sv = device_view(src_v_cache, dev);
+  const void *pr = device_view(block_pairs, dev);
+  if (!dk || !dv || !sk || !sv || !pr) return PA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  pa::copy_blocks_kernel<<<2 * num_pairs, pa::kCacheThreads, 0, st>>>(
+      static_cast<uint4 *>(const_cast<void *>(dk)), static_cast<uint4 *>(const_cast<void *>(dv)),
+      static_cast<const uint4 *>(sk), static_cast<const uint4 *>(sv),
+      static_cast<const int64_t *>(pr), static_cast<int64_t>(block_bytes / 16), src_num_blocks,
+      dst_num_blocks);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -122,3 +122,18 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libpa.so"))
     with pytest.raises(_lib.LibraryNotBuilt):
         _lib.lib()
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(n=0), OK),
+    (dict(pairs=None), INVALID),
+    (dict(dk=None), INVALID),
+    (dict(bb=24), INVALID),
+    (dict(sk=FAKE + 4), INVALID),
+    (dict(snb=0), INVALID),
+])
+def test_swap_rejects_bad_arguments_on_host(kw, expect):
+    a = dict(dk=FAKE, dv=FAKE, sk=FAKE, sv=FAKE, pairs=FAKE, n=3, bb=4096, snb=8,
+             dnb=8, stream=None)
+    a.update(kw)
+    assert _lib.lib().pa_swap_blocks(*a.values()) == expect

@@ -224,3 +224,150 @@ def test_random_operations_keep_invariants(seed):
             if cow:
                 assert before[L0 // B] == cow[0] and after[L0 // B] == cow[1]
         assert_invariants(pool, live)
+
+
+def test_swap_out_and_in_keeps_both_pools_consistent():
+    """Preemption by swapping ([Day28] §六 question 4, FAQ Q3): the swapped
+    sequence takes private CPU copies; blocks still shared stay on the GPU."""
+    gpu, cpu = BlockPool(12, shuffle_seed=1), BlockPool(8)
+    gpu.add_seq(1)
+    gpu.append(1, 40)              # 3 blocks
+    gpu.fork(1, 2)                 # seq 2 shares all three
+    gpu.append(2, 1)               # CoW of the partial last block
+    before = tables_of(gpu, [1])[2][0]
+    free_gpu = gpu.num_free
+    pairs = gpu.swap_out(cpu, 1)
+    assert [int(a) for a in pairs[:, 0]] == before
+    assert cpu.seq_len(1) == 40 and gpu.seq_len(1) == -1
+    assert cpu.num_free == 8 - 3
+    # blocks 0,1 still shared with seq 2 stay; the old last block is freed
+    assert gpu.num_free == free_gpu + 1
+    assert_invariants(gpu, [2])
+    assert_invariants(cpu, [1])
+    assert tables_of(cpu, [1])[2][0] == [int(b) for b in pairs[:, 1]]
+    back = gpu.swap_in(cpu, 1)
+    assert [int(a) for a in back[:, 0]] == [int(b) for b in pairs[:, 1]]
+    assert cpu.num_free == 8 and gpu.seq_len(1) == 40
+    assert_invariants(gpu, [1, 2])
+    assert tables_of(gpu, [1])[2][0] == [int(b) for b in back[:, 1]]
+
+
+def test_swap_errors_change_nothing():
+    gpu, cpu = BlockPool(10), BlockPool(2)
+    gpu.add_seq(0)
+    gpu.append(0, 48)              # 3 blocks, more than the CPU pool holds
+    with pytest.raises(PagedAttentionError) as e:
+        gpu.swap_out(cpu, 0)
+    assert e.value.status == 5
+    assert gpu.seq_len(0) == 48 and cpu.num_free == 2 and gpu.num_free == 7
+    with pytest.raises(PagedAttentionError) as e:
+        gpu.swap_out(cpu, 9)
+    assert e.value.status == 6
+    cpu.add_seq(0)
+    with pytest.raises(PagedAttentionError) as e:
+        gpu.swap_out(cpu, 0)       # id already present in the destination
+    assert e.value.status == 1
+
+
+# ------------------------------------------------ automatic prefix caching
+
+def test_prefix_caching_shares_whole_blocks_of_a_common_prompt():
+    """Two requests with the same 1000-token system prompt ([Ch7] §7.1
+    前缀共享; [Day28] §六 question 2): the second finds the first 62 full
+    blocks (992 tokens) cached and gets slot -1 for them; the block holding
+    prompt tokens 992-999 differs (other suffix) and is its own."""
+    rng = np.random.default_rng(0)
+    prompt = rng.integers(0, 32000, 1000)
+    pool = BlockPool(200, shuffle_seed=3)
+    pool.enable_prefix_caching()
+    pool.add_seq(0)
+    s0, _, c0 = pool.append_tokens(0, np.concatenate([prompt, rng.integers(0, 32000, 50)]))
+    pool.add_seq(1)
+    s1, _, c1 = pool.append_tokens(1, np.concatenate([prompt, rng.integers(0, 32000, 70)]))
+    assert c0 == 0 and c1 == 992
+    assert np.all(s1[:992] == -1) and np.all(s1[992:] >= 0)
+    rows = tables_of(pool, [0, 1])[2]
+    assert rows[0][:62] == rows[1][:62] and rows[0][62] != rows[1][62]
+    assert all(pool.refcount(b) == 2 for b in rows[0][:62])
+    # slots of the non-cached tokens follow the table
+    for i in range(992, 1070):
+        assert s1[i] == oracle.slot(rows[1], i, B)
+    assert_invariants(pool, [0, 1])
+
+
+def test_prefix_cache_survives_its_owner_and_is_evicted_last():
+    rng = np.random.default_rng(1)
+    prompt = rng.integers(0, 32000, 160)          # 10 full blocks
+    pool = BlockPool(16)
+    pool.enable_prefix_caching()
+    pool.add_seq(0)
+    pool.append_tokens(0, prompt)
+    pool.free_seq(0)
+    assert pool.num_free == 16 and pool.num_cached == 10
+    pool.add_seq(1)
+    _, _, c = pool.append_tokens(1, prompt)       # all found again
+    assert c == 160 and pool.num_free == 6
+    pool.free_seq(1)
+    # a request that needs 13 fresh blocks evicts the 7 least recently freed;
+    # blocks are freed last-first, so the prompt's tail goes, its head stays
+    pool.add_seq(2)
+    _, _, c = pool.append_tokens(2, rng.integers(0, 32000, 13 * 16))
+    assert c == 0 and pool.num_cached == 10 - 7 + 13
+    pool.add_seq(3)
+    with pytest.raises(PagedAttentionError) as e:   # 3 cached + 7 fresh > 3 left
+        pool.append_tokens(3, prompt)
+    assert e.value.status == 5 and pool.seq_len(3) == 0
+    pool.free_seq(2)
+    _, _, c = pool.append_tokens(3, prompt)
+    assert c == 3 * 16                              # the surviving head
+    assert_invariants(pool, [3])
+
+
+def test_prefix_cache_matches_only_an_identical_prefix():
+    rng = np.random.default_rng(2)
+    a = rng.integers(0, 32000, 64)
+    b = a.copy()
+    b[20] += 1                                    # differs inside block 1
+    pool = BlockPool(20)
+    pool.enable_prefix_caching()
+    pool.add_seq(0)
+    pool.append_tokens(0, a)
+    pool.add_seq(1)
+    _, _, c = pool.append_tokens(1, b)
+    assert c == 16                                # block 0 only; then a miss
+    pool.add_seq(2)
+    _, _, c = pool.append_tokens(2, np.concatenate([a[16:32], a[:16], a[32:]]))
+    assert c == 0                                 # same tokens, other order
+
+
+def test_prefix_caching_with_incremental_decode_and_fork():
+    rng = np.random.default_rng(3)
+    toks = rng.integers(0, 32000, 40)
+    pool = BlockPool(30)
+    pool.enable_prefix_caching()
+    pool.add_seq(0)
+    pool.append_tokens(0, toks[:10])
+    for t in toks[10:]:                           # one token per decode step
+        pool.append_tokens(0, [t])
+    pool.fork(0, 1)                               # shares the partial block too
+    _, cow, _ = pool.append_tokens(1, [5])
+    assert cow is not None                        # writer copies the shared block
+    pool.add_seq(2)
+    _, _, c = pool.append_tokens(2, toks)
+    assert c == 32                                # the two blocks filled step by step
+    assert_invariants(pool, [0, 1, 2])
+
+
+def test_disabling_prefix_caching_forgets_keys():
+    pool = BlockPool(8)
+    pool.enable_prefix_caching()
+    pool.add_seq(0)
+    pool.append_tokens(0, list(range(32)))
+    pool.free_seq(0)
+    assert pool.num_cached == 2
+    pool.enable_prefix_caching(False)
+    assert pool.num_cached == 0 and pool.num_free == 8
+    pool.enable_prefix_caching()
+    pool.add_seq(1)
+    _, _, c = pool.append_tokens(1, list(range(32)))
+    assert c == 0
