@@ -449,12 +449,93 @@ def run_reference(args, world, rank):
     }
 
 
+# ------------------------------------------------------- other operations
+
+def run_loop(args):
+    """Continuous-batching decode loop (requests join and leave each step;
+    preemption by swapping): decode tokens/s over the whole loop, host work
+    included, and KV utilisation of the paged pool vs max-length reservation."""
+    from paged_kv_cache_429_b200.serve_loop import DecodeLoop, LoopConfig
+    cfg = LoopConfig(num_q_heads=32, num_kv_heads=32, head_dim=128, num_blocks=16384,
+                     cpu_blocks=8192, max_num_seqs=256, max_model_len=4096,
+                     prompt_median=600, prompt_sigma=0.7, output_median=300,
+                     output_sigma=0.7, arrivals_per_step=4.0, watermark_blocks=64,
+                     seed=args.seed)
+    loop = DecodeLoop(cfg)
+    loop.run(args.warmup)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    stats = loop.run(args.steps)
+    torch.cuda.synchronize()
+    secs = time.perf_counter() - t0
+    live = [st for st in stats if st["running"]]
+    tokens = sum(st["running"] for st in live)
+    mean = lambda k: sum(st[k] for st in live) / max(len(live), 1)
+    return {
+        "op": "loop", "metric": "continuous-batching decode loop: decode tokens/s "
+        "(one attention layer, host scheduling included)",
+        "value": round(tokens / secs, 1), "unit": "tokens/s", "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 4),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "32/32 heads, d128, bf16, pool 16384 blocks, "
+                   "max_num_seqs 256, max_model_len 4096, prompts lognormal(600), "
+                   "outputs lognormal(300), Poisson arrivals 4/step", "seed": args.seed},
+        "mean_running": round(mean("running"), 1),
+        "kv_utilisation_paged": round(mean("paged_util"), 4),
+        "kv_utilisation_reserved_max_len": round(mean("reserved_util"), 4),
+        "min_kv_utilisation_paged": round(min(st["paged_util"] for st in live), 4),
+        "preemptions": loop.preemptions, "finished": loop.finished,
+    }
+
+
+def run_swap(args):
+    """Swap-out of whole sequences to pinned host memory and back in."""
+    from paged_kv_cache_429_b200 import BlockPool, pa_swap_blocks
+    from paged_kv_cache_429_b200.batch import DecodeBatch
+    w = synth.WORKLOADS["llama7b"]
+    b = DecodeBatch.build(w, args.seed)
+    b.k_old = b.v_old = None
+    seqs = list(range(16))
+    nblk = sum(b.pool.seq_num_blocks(s) for s in seqs)
+    cpu = BlockPool(nblk)
+    hk = torch.empty((nblk,) + tuple(b.k_cache.shape[1:]), dtype=b.k_cache.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = np.concatenate([b.pool.swap_out(cpu, s) for s in seqs])
+    in_pairs = np.concatenate([b.pool.swap_in(cpu, s) for s in seqs])
+    po, pi = torch.from_numpy(out_pairs).cuda(), torch.from_numpy(in_pairs).cuda()
+    block_bytes = b.k_cache[0].numel() * b.k_cache.element_size()
+    moved = 2 * block_bytes * len(out_pairs)
+    times = {"out": [], "in": []}
+    for it in range(args.warmup + args.steps):
+        for d, (dk, dv, sk, sv, pr) in (("out", (hk, hv, b.k_cache, b.v_cache, po)),
+                                         ("in", (b.k_cache, b.v_cache, hk, hv, pi))):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            pa_swap_blocks(dk, dv, sk, sv, pr)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                times[d].append(e0.elapsed_time(e1))
+    gbs = {d: moved / (statistics.median(t) * 1e-3) / 1e9 for d, t in times.items()}
+    return {
+        "op": "swap", "metric": "pa_swap_blocks GB/s (device <-> pinned host), one launch",
+        "value": round(min(gbs.values()), 2), "unit": "GB/s",
+        "swap_out_gbs": round(gbs["out"], 2), "swap_in_gbs": round(gbs["in"], 2),
+        "bytes_per_direction": moved, "blocks": len(out_pairs), "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "data": "synthetic",
+        "config": {"workload": "16 sequences of the llama7b workload (32 KV heads, d128, bf16)"},
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["step", "loop", "swap"], default="step",
+                    help="step: the decode step (default); loop: continuous batching; "
+                         "swap: block swapping to host memory")
     ap.add_argument("--workload", default="llama7b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--partition-size", type=int, default=None)
     ap.add_argument("--seed", type=int, default=0)
@@ -470,6 +551,11 @@ def main(argv=None):
         line = run_reference(args, world, rank)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return
+    if args.op != "step":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        line = run_loop(args) if args.op == "loop" else run_swap(args)
+        print(json.dumps(line), flush=True)
         return
     world, rank, local = init_dist()
     if args.gpus != world and world > 1:

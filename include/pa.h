@@ -282,6 +282,16 @@ PA_API pa_status pa_pool_append(pa_pool *pool, int64_t seq_id, int n_tokens,
                          int64_t *slots_out, int64_t *cow_pairs_out,
                          int *n_cow_out);
 
+/* One decode step for n sequences at once (continuous batching, [Ch7]
+ * §7.1, [Day28] §五): append one token to each of seq_ids[0..n) (distinct),
+ * writing its slot to slots_out[i]. Shared partly filled last blocks are
+ * copied first; those (old, new) pairs go to cow_pairs_out [n][2] and their
+ * count to *n_cow_out. PA_ERR_OUT_OF_BLOCKS (the pool cannot cover every
+ * new block) changes nothing. */
+PA_API pa_status pa_pool_append_decode(pa_pool *pool, const int64_t *seq_ids, int n,
+                                       int64_t *slots_out, int64_t *cow_pairs_out,
+                                       int *n_cow_out);
+
 /* Drop a sequence: every block's refcount - 1; blocks reaching 0 return to
  * the free list ([Day28] §五: a finished request returns its blocks). */
 PA_API pa_status pa_pool_free_seq(pa_pool *pool, int64_t seq_id);

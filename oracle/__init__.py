@@ -282,3 +282,34 @@ def check_block_tables(block_tables, context_lens, num_blocks: int,
     if num_free is not None and num_free + len(uses) != num_blocks:
         errors.append(f"{num_free} free + {len(uses)} used != {num_blocks}")
     return errors
+
+
+# ------------------------------------------------- utilisation (plain defs)
+
+def paged_utilisation(context_lens, block_size: int = 16) -> float:
+    """Tokens stored / token slots of the blocks held: sum L / (B sum ceil(L/B)).
+    Only the last, partly filled block of each sequence wastes slots
+    ([Day28] §4.2: internal fragmentation confined to the last block)."""
+    lens = [int(x) for x in context_lens]
+    held = sum(-(-L // block_size) for L in lens) * block_size
+    return sum(lens) / held if held else 1.0
+
+
+def reserved_utilisation(context_lens, reserve_tokens: int) -> float:
+    """Tokens stored / slots reserved when every running request holds a
+    contiguous region of its maximum length ([Ch7] §7.1, [OSPage] §服务化痛点,
+    [Day28] §4.1: preallocation by max_seq_len)."""
+    lens = [int(x) for x in context_lens]
+    return sum(lens) / (len(lens) * reserve_tokens) if lens else 1.0
+
+
+def reserved_waste_bytes(reserve_tokens: int, used_tokens: int,
+                         bytes_per_token: int) -> int:
+    """Bytes of a contiguous reservation that were never used ([Day28] §4.1
+    worked example: 2048 reserved, 400 used)."""
+    return (reserve_tokens - used_tokens) * bytes_per_token
+
+
+def effective_capacity(kv_bytes: float, utilisation: float) -> float:
+    """Usable KV bytes = bytes given to KV x utilisation ([Ch7] §7.3 例 7-3)."""
+    return kv_bytes * utilisation

@@ -235,6 +235,20 @@ class BlockPool:
             "pa_pool_append")
         return slots, ((int(pair[0]), int(pair[1])) if ncow.value else None)
 
+    def append_decode(self, seq_ids):
+        """One token for each listed sequence. Returns (slots int64[n],
+        cow pairs int64[k][2])."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = np.empty(n, dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int64)
+        ncow = ctypes.c_int(0)
+        _ok(self._lib.pa_pool_append_decode(self._h, ids.ctypes.data if n else None, n,
+                                            slots.ctypes.data if n else None,
+                                            pairs.ctypes.data, ctypes.byref(ncow)),
+            "pa_pool_append_decode")
+        return slots, pairs[:ncow.value]
+
     def enable_prefix_caching(self, enable: bool = True) -> None:
         _ok(self._lib.pa_pool_enable_prefix_caching(self._h, int(enable)),
             "pa_pool_enable_prefix_caching")

@@ -40,6 +40,7 @@ SIGNATURES = {
     "pa_pool_add_seq": (_i32, [_vp, _i64]),
     "pa_pool_fork": (_i32, [_vp, _i64, _i64]),
     "pa_pool_append": (_i32, [_vp, _i64, _i32, _vp, _vp, ctypes.POINTER(_i32)]),
+    "pa_pool_append_decode": (_i32, [_vp, _vp, _i32, _vp, _vp, ctypes.POINTER(_i32)]),
     "pa_pool_free_seq": (_i32, [_vp, _i64]),
     "pa_pool_block_tables": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp]),
     "pa_pool_enable_prefix_caching": (_i32, [_vp, _i32]),

@@ -219,6 +219,48 @@ pa_status pa_pool_append(pa_pool *pool, int64_t seq_id, int n_tokens,
   return PA_OK;
 }
 
+pa_status pa_pool_append_decode(pa_pool *pool, const int64_t *seq_ids, int n,
+                                int64_t *slots_out, int64_t *cow_pairs_out, int *n_cow_out) {
+  if (!pool || n < 0 || !n_cow_out || (n > 0 && (!seq_ids || !slots_out || !cow_pairs_out)))
+    return PA_ERR_INVALID_ARG;
+  *n_cow_out = 0;
+  const int64_t B = pool->block_size;
+  // all-or-nothing: find every sequence and count the blocks needed first
+  std::vector<Sequence *> seqs(n);
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    auto it = pool->seqs.find(seq_ids[i]);
+    if (it == pool->seqs.end()) return PA_ERR_NOT_FOUND;
+    Sequence &s = it->second;
+    seqs[i] = &s;
+    if (s.len % B == 0) ++need;                                     // new block
+    else if (pool->refcount[s.blocks.back()] > 1) ++need;           // copy-on-write
+  }
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j)
+      if (seqs[i] == seqs[j]) return PA_ERR_INVALID_ARG;            // listed twice
+  if (need > pool->available()) return PA_ERR_OUT_OF_BLOCKS;
+  for (int i = 0; i < n; ++i) {
+    Sequence &s = *seqs[i];
+    s.keyed = false;
+    s.pending.clear();
+    if (s.len % B == 0) {
+      s.blocks.push_back(pool->take());
+    } else if (pool->refcount[s.blocks.back()] > 1) {
+      const int32_t old_b = s.blocks.back();
+      const int32_t new_b = pool->take();
+      pool->release(old_b);
+      s.blocks.back() = new_b;
+      cow_pairs_out[2 * *n_cow_out] = old_b;
+      cow_pairs_out[2 * *n_cow_out + 1] = new_b;
+      ++*n_cow_out;
+    }
+    slots_out[i] = static_cast<int64_t>(s.blocks.back()) * B + s.len % B;
+    s.len += 1;
+  }
+  return PA_OK;
+}
+
 pa_status pa_pool_free_seq(pa_pool *pool, int64_t seq_id) {
   if (!pool) return PA_ERR_INVALID_ARG;
   auto it = pool->seqs.find(seq_id);

@@ -414,3 +414,43 @@ def test_reshape_bf16_copies_bits_and_skips_negative_slots():
     assert np.count_nonzero(kc) == np.count_nonzero(key[[0, 2]])
     with pytest.raises(ValueError):
         oracle.reshape_and_cache(key, val, kc, vc, np.array([64, 0, 0]), oracle.KV_BF16)
+
+
+# ------------------------------------------------------------ utilisation
+
+def read_golden_kv(path):
+    out = {}
+    for row in read_golden_rows(path):
+        out[row[0]] = float(row[1])
+    return out
+
+
+def test_capacity_and_waste_worked_examples(golden_dir):
+    g = read_golden_kv(os.path.join(golden_dir, "utilisation_examples.txt"))
+    old = oracle.effective_capacity(g["capacity_kv_gb"], g["capacity_u_old"])
+    new = oracle.effective_capacity(g["capacity_kv_gb"], g["capacity_u_new"])
+    assert old == pytest.approx(g["capacity_eff_old_gb"])
+    assert new == pytest.approx(g["capacity_eff_new_gb"])
+    assert new / old == pytest.approx(g["capacity_gain"])
+    waste = oracle.reserved_waste_bytes(int(g["reserve_tokens"]), int(g["used_tokens"]),
+                                        int(g["llama7b_bytes_per_token"]))
+    assert waste == int(g["unused_bytes"])
+    assert int(g["reserve_tokens"]) - int(g["used_tokens"]) == int(g["unused_tokens"])
+    # the per-token figure itself is the KV-size formula for Llama-7B fp16
+    assert oracle.kv_bytes_per_token(32, 32, 128, 2) == int(g["llama7b_bytes_per_token"])
+
+
+def test_paged_utilisation_closed_forms():
+    assert oracle.paged_utilisation([16, 32, 160]) == 1.0
+    assert oracle.paged_utilisation([1]) == 1 / 16
+    assert oracle.paged_utilisation([17, 15]) == 32 / 48
+    # the waste bound: at most 15 unused slots per sequence
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        lens = rng.integers(1, 5000, size=rng.integers(1, 40))
+        u = oracle.paged_utilisation(lens)
+        held = sum(-(-int(L) // 16) * 16 for L in lens)
+        assert held - sum(lens) <= 15 * len(lens)
+        assert u >= 1 - 15 * len(lens) / held
+    assert oracle.reserved_utilisation([400], 2048) == 400 / 2048
+    assert oracle.reserved_utilisation([1024, 2048], 2048) == 0.75

@@ -371,3 +371,28 @@ def test_disabling_prefix_caching_forgets_keys():
     pool.add_seq(1)
     _, _, c = pool.append_tokens(1, list(range(32)))
     assert c == 0
+
+
+def test_append_decode_one_token_each():
+    pool = BlockPool(12, shuffle_seed=4)
+    for sid, n in ((1, 16), (2, 5), (3, 31)):
+        pool.add_seq(sid)
+        pool.append(sid, n)
+    pool.fork(2, 4)                                  # 4 shares 2's partial block
+    free0 = pool.num_free
+    slots, cow = pool.append_decode([1, 2, 3, 4])
+    # 2 writes first and copies; 4 is then the only owner and writes in place
+    assert len(cow) == 1
+    assert pool.num_free == free0 - 2                # seq 1's new block + 2's copy
+    rows = tables_of(pool, [1, 2, 3, 4])[2]
+    for sl, sid, row in zip(slots, (1, 2, 3, 4), rows):
+        assert sl == oracle.slot(row, pool.seq_len(sid) - 1, B)
+    assert_invariants(pool, [1, 2, 3, 4])
+    with pytest.raises(PagedAttentionError):
+        pool.append_decode([1, 1])                   # listed twice
+    small = BlockPool(1)
+    small.add_seq(0)
+    small.append(0, 16)
+    with pytest.raises(PagedAttentionError) as e:
+        small.append_decode([0])
+    assert e.value.status == 5 and small.seq_len(0) == 16
