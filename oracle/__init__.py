@@ -75,6 +75,9 @@ def _load():
     lib.oracle_reshape_and_cache.restype = i32
     lib.oracle_copy_blocks.argtypes = [vp, vp, vp, i32, i64, i32]
     lib.oracle_copy_blocks.restype = i32
+    lib.oracle_paged_prefill.argtypes = [vp, vp, vp, vp, i32, f64, f64, vp, i32, vp,
+                                         vp, i32, i32, i32, i32, i32, i32, f64]
+    lib.oracle_paged_prefill.restype = i32
     lib.oracle_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32]
     lib.oracle_swap_blocks.restype = i32
     lib.oracle_paged_decode.argtypes = [vp, vp, vp, vp, i32, f64, f64, vp, i32,
@@ -240,6 +243,30 @@ def paged_decode_split(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
         _ptr(np.ascontiguousarray(v_cache)), kv_dtype, k_scale, v_scale,
         _ptr(bt), bt.shape[1], _ptr(cl), S, Hq, Hkv, D, B, NB, sm_scale,
         partition_size), "paged_decode_split")
+    return out
+
+
+def paged_prefill(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                  block_tables: np.ndarray, query_start: np.ndarray,
+                  context_lens: np.ndarray, sm_scale: float,
+                  kv_dtype: int = KV_BF16, k_scale: float = 1.0,
+                  v_scale: float = 1.0) -> np.ndarray:
+    """fp64 causal chunked-prefill attention; q / out are [T][Hq][D] with
+    sequence s's rows query_start[s] .. query_start[s+1]-1."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    qs = np.ascontiguousarray(query_start, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    T, Hq, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    assert Dc == D and qs.size == cl.size + 1 and qs[-1] == T
+    k_scale, v_scale = float(np.float32(k_scale)), float(np.float32(v_scale))
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    _check(_load().oracle_paged_prefill(
+        _ptr(out), _ptr(q), _ptr(np.ascontiguousarray(k_cache)),
+        _ptr(np.ascontiguousarray(v_cache)), kv_dtype, k_scale, v_scale, _ptr(bt),
+        bt.shape[1], _ptr(qs), _ptr(cl), cl.size, Hq, Hkv, D, B, NB, sm_scale),
+        "paged_prefill")
     return out
 
 

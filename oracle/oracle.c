@@ -409,3 +409,74 @@ int oracle_paged_decode_split(double *out, const uint16_t *q,
   }
   return 0;
 }
+
+/* Chunked prefill attention through block tables. Sequence s holds
+ * context_lens[s] tokens in the cache; its last n_s = query_start[s+1] -
+ * query_start[s] tokens are this chunk's queries (rows query_start[s] ..
+ * query_start[s+1]-1 of q and out). The query at position p attends to the
+ * keys at positions 0..p (causal):
+ *   z_t = sm_scale * q . K_t (t <= p),  out = sum_t softmax(z)_t V_t.
+ * Prefill KV is written block-wise into the same pool ([Day28] FAQ Q4,
+ * chunked prefill mixes prompt chunks with decode), so a chunk attends to
+ * the cached prefix and to itself. Two-pass softmax in double. */
+int oracle_paged_prefill(double *out, const uint16_t *q, const void *k_cache,
+                         const void *v_cache, int kv_dtype, double k_scale,
+                         double v_scale, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *query_start,
+                         const int32_t *context_lens, int num_seqs,
+                         int num_q_heads, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, double sm_scale) {
+  int group, s;
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return 1;
+  group = num_q_heads / num_kv_heads;
+  for (s = 0; s < num_seqs; ++s) {
+    int L = context_lens[s];
+    int q0 = query_start[s], n = query_start[s + 1] - query_start[s];
+    const int32_t *bt_row = block_tables + (int64_t)s * max_blocks_per_seq;
+    int h, i, t, d;
+    double *Kc, *Vc, *z;
+    if (n < 0 || n > L || (L + block_size - 1) / block_size > max_blocks_per_seq) return 1;
+    if (L == 0) continue;
+    Kc = (double *)malloc(sizeof(double) * (size_t)L * head_dim);
+    Vc = (double *)malloc(sizeof(double) * (size_t)L * head_dim);
+    z = (double *)malloc(sizeof(double) * (size_t)L);
+    if (!Kc || !Vc || !z) {
+      free(Kc); free(Vc); free(z);
+      return 2;
+    }
+    for (h = 0; h < num_kv_heads; ++h) {
+      if (gather_kv(Kc, Vc, k_cache, v_cache, kv_dtype, k_scale, v_scale, bt_row, L,
+                    h, num_kv_heads, head_dim, block_size, num_blocks)) {
+        free(Kc); free(Vc); free(z);
+        return 1;
+      }
+      for (i = 0; i < n; ++i) {
+        int p = L - n + i, g;
+        for (g = 0; g < group; ++g) {
+          int hq = h * group + g;
+          const uint16_t *qv = q + ((int64_t)(q0 + i) * num_q_heads + hq) * head_dim;
+          double *o = out + ((int64_t)(q0 + i) * num_q_heads + hq) * head_dim;
+          double zmax = -INFINITY, denom = 0.0;
+          for (t = 0; t <= p; ++t) {
+            double acc = 0.0;
+            for (d = 0; d < head_dim; ++d)
+              acc += bf16_bits_to_double(qv[d]) * Kc[(int64_t)t * head_dim + d];
+            z[t] = sm_scale * acc;
+            if (z[t] > zmax) zmax = z[t];
+          }
+          for (t = 0; t <= p; ++t) {
+            z[t] = exp(z[t] - zmax);
+            denom += z[t];
+          }
+          for (d = 0; d < head_dim; ++d) o[d] = 0.0;
+          for (t = 0; t <= p; ++t) {
+            double w = z[t] / denom;
+            for (d = 0; d < head_dim; ++d) o[d] += w * Vc[(int64_t)t * head_dim + d];
+          }
+        }
+      }
+    }
+    free(Kc); free(Vc); free(z);
+  }
+  return 0;
+}

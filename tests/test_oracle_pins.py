@@ -454,3 +454,78 @@ def test_paged_utilisation_closed_forms():
         assert u >= 1 - 15 * len(lens) / held
     assert oracle.reserved_utilisation([400], 2048) == 400 / 2048
     assert oracle.reserved_utilisation([1024, 2048], 2048) == 0.75
+
+
+# ---------------------------------------------------------------- prefill
+
+def numpy_prefill(q, kc, vc, bt, qs, lens, scale, B=16):
+    """Test-local second formulation: per sequence a [n x L] score matrix
+    with an explicit causal mask, row softmax, times V."""
+    T, Hq, D = q.shape
+    Hkv = kc.shape[1]
+    g = Hq // Hkv
+    out = np.zeros((T, Hq, D))
+    qf, kf, vf = bits_to_f64(q), bits_to_f64(kc), bits_to_f64(vc)
+    for s in range(len(lens)):
+        L, q0, n = int(lens[s]), int(qs[s]), int(qs[s + 1] - qs[s])
+        pos = np.arange(L)
+        qpos = L - n + np.arange(n)
+        mask = pos[None, :] <= qpos[:, None]
+        for hq in range(Hq):
+            K = kf[bt[s][pos // B], hq // g, pos % B]
+            V = vf[bt[s][pos // B], hq // g, pos % B]
+            Z = scale * (qf[q0:q0 + n, hq] @ K.T)
+            Z = np.where(mask, Z, -np.inf)
+            W = np.exp(Z - Z.max(axis=1, keepdims=True))
+            out[q0:q0 + n, hq] = (W / W.sum(axis=1, keepdims=True)) @ V
+    return out
+
+
+def prefill_case(rng, lens, chunks, Hq, Hkv, D, NB):
+    q_total = sum(chunks)
+    q = bf16_bits(rng.standard_normal((q_total, Hq, D)))
+    _, kc, vc, bt, lens = make_case(rng, len(lens), Hq, Hkv, D, lens, NB)
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    return q, kc, vc, bt, qs, lens
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_prefill_against_numpy_formulation(seed):
+    rng = np.random.default_rng(40 + seed)
+    lens, chunks = [37, 5, 64, 100], [37, 5, 20, 1]   # full, full, chunked, decode-like
+    q, kc, vc, bt, qs, lens = prefill_case(rng, lens, chunks, 4, 2, 16, 40)
+    out = oracle.paged_prefill(q, kc, vc, bt, qs, lens, 0.25)
+    ref = numpy_prefill(q, kc, vc, bt, qs, lens, 0.25)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_prefill_against_torch_sdpa_causal():
+    """A whole prompt (no cached prefix) is causal attention."""
+    rng = np.random.default_rng(42)
+    q, kc, vc, bt, qs, lens = prefill_case(rng, [70], [70], 4, 4, 64, 8)
+    out = oracle.paged_prefill(q, kc, vc, bt, qs, lens, 0.125)
+    pos = np.arange(70)
+    K = torch.from_numpy(bits_to_f64(kc)[bt[0][pos // 16], :, pos % 16]).permute(1, 0, 2)
+    V = torch.from_numpy(bits_to_f64(vc)[bt[0][pos // 16], :, pos % 16]).permute(1, 0, 2)
+    Q = torch.from_numpy(bits_to_f64(q)).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=0.125)
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_chunk_of_one_token_is_decode():
+    rng = np.random.default_rng(43)
+    lens = [33, 80, 1]
+    q, kc, vc, bt, qs, lens = prefill_case(rng, lens, [1, 1, 1], 8, 2, 64, 20)
+    pre = oracle.paged_prefill(q, kc, vc, bt, qs, lens, 0.125)
+    dec = oracle.paged_decode(q, kc, vc, bt, lens, 0.125)
+    np.testing.assert_array_equal(pre, dec)
+
+
+def test_prefill_chunks_compose():
+    """Prefilling a prompt in two chunks gives the rows of one whole pass."""
+    rng = np.random.default_rng(44)
+    q, kc, vc, bt, qs, lens = prefill_case(rng, [90], [90], 2, 2, 64, 8)
+    whole = oracle.paged_prefill(q, kc, vc, bt, qs, lens, 0.125)
+    first = oracle.paged_prefill(q[:50], kc, vc, bt, np.array([0, 50]), [50], 0.125)
+    second = oracle.paged_prefill(q[50:], kc, vc, bt, np.array([0, 40]), [90], 0.125)
+    np.testing.assert_array_equal(np.concatenate([first, second]), whole)
