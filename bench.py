@@ -527,13 +527,60 @@ def run_swap(args):
     }
 
 
+def run_prefill(args):
+    """Chunked prefill attention: 16 whole 2048-token prompts, 32 query /
+    8 KV heads, d128, bf16 KV (the prompts' K/V already in the cache)."""
+    from paged_kv_cache_429_b200 import pa_prefill
+    from paged_kv_cache_429_b200.batch import DecodeBatch
+    S, Hq, Hkv, D, L = 16, 32, 8, 128, 2048
+    w = synth.Workload("prefill", S, Hq, Hkv, D, False, pool_factor=1.2)
+    b = DecodeBatch.build(w, args.seed, lens=np.full(S, L))
+    b.run_ops(b.step_ops)
+    b.k_old = b.v_old = None
+    q = synth.randn_bf16((S * L, Hq, D), args.seed, w.name, "q_prefill", "cuda")
+    qs = torch.arange(0, S * L + 1, L, dtype=torch.int32, device="cuda")
+    out = torch.empty((S * L, Hq, D), dtype=torch.float32, device="cuda")
+    flops = S * Hq * 4 * D * (L * (L + 1) // 2)
+    def once():
+        pa_prefill(out, q, b.k_cache, b.v_cache, b.block_tables, qs, b.context_lens, L, L,
+                   w.sm_scale)
+    for _ in range(args.warmup):
+        once()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        e0.record()
+        once()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(c) for a, c in evs)
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak = 1672.3
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return {
+        "op": "prefill", "metric": "chunked prefill attention TFLOP/s (causal, QK and PV)",
+        "value": round(tflops, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{S} whole {L}-token prompts, {Hq}/{Hkv} heads, d{D}, bf16 KV"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                     "kernel": "paged_prefill_kernel (warp-level mma.sync)"},
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["step", "loop", "swap"], default="step",
+    ap.add_argument("--op", choices=["step", "loop", "swap", "prefill"], default="step",
                     help="step: the decode step (default); loop: continuous batching; "
                          "swap: block swapping to host memory")
     ap.add_argument("--workload", default="llama7b", choices=sorted(synth.WORKLOADS))
@@ -554,7 +601,7 @@ def main(argv=None):
         return
     if args.op != "step":
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        line = run_loop(args) if args.op == "loop" else run_swap(args)
+        line = {"loop": run_loop, "swap": run_swap, "prefill": run_prefill}[args.op](args)
         print(json.dumps(line), flush=True)
         return
     world, rank, local = init_dist()

@@ -170,6 +170,30 @@ PA_API pa_status pa_decode_no_alloc(float *out, const void *q, const void *k_cac
                                     int num_blocks, float sm_scale,
                                     int partition_size, void *stream);
 
+/* Chunked prefill attention through block tables (bf16 caches).
+ * Prefill KV is written block-wise into the same pool, and long prompts are
+ * prefilled in chunks ([Day28] FAQ Q4). Sequence s holds L = context_lens[s]
+ * tokens in the cache (its K/V already written, pa_reshape_and_cache); its
+ * last n_s = query_start[s+1] - query_start[s] tokens are this call's
+ * queries, rows query_start[s] .. query_start[s+1]-1 of q and out. The query
+ * at position p = L - n_s + i attends causally to keys 0..p:
+ *     out[row][hq] = sum_{t<=p} softmax_t(sm_scale * q[row][hq] . K_t) V_t.
+ *   out          fp32 [num_tokens][num_q_heads][head_dim], 16-byte aligned.
+ *   q            bf16 [num_tokens][num_q_heads][head_dim].
+ *   query_start  int32 [num_seqs + 1], device; query_start[0] = 0,
+ *                query_start[num_seqs] = num_tokens, n_s <= L.
+ *   max_query_len  host-known bound of every n_s (sizes the grid).
+ *   Other arguments as for pa_decode. fp8 caches: PA_ERR_UNSUPPORTED. */
+PA_API pa_status pa_prefill(float *out, const void *q, const void *k_cache,
+                            const void *v_cache, pa_kv_dtype kv_dtype,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *query_start,
+                            const int32_t *context_lens, int max_query_len,
+                            int max_context_len, int num_seqs, int num_tokens,
+                            int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int num_blocks, float sm_scale,
+                            void *stream);
+
 /* ------------------------------------------------------- cache writes ---- */
 
 /* Scatter new tokens' K/V into their cache slots: for token t and KV head

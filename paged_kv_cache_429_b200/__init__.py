@@ -5,6 +5,7 @@ of libpa.so; PyTorch is used for device memory, streams and dtypes. The
 functions carry the names of the C entry points (include/pa.h):
 
     pa_decode               decode-step attention through block tables
+    pa_prefill              chunked causal prefill attention through block tables
     pa_reshape_and_cache    scatter new K/V into cache slots (bf16 / fp8)
     pa_copy_blocks          copy-on-write block copies
     pa_swap_blocks          block copies between the GPU cache and pinned host memory
@@ -28,7 +29,7 @@ from ._lib import STATUS_NAMES, LibraryNotBuilt
 
 __all__ = [
     "PA_KV_BF16", "PA_KV_FP8_E4M3", "BLOCK_SIZE", "PagedAttentionError",
-    "LibraryNotBuilt", "pa_decode", "pa_reshape_and_cache", "pa_copy_blocks",
+    "LibraryNotBuilt", "pa_decode", "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks",
     "pa_swap_blocks", "pa_decode_workspace_size", "pa_get_device_error",
     "pa_status_string",
     "BlockPool", "kv_dtype_of",
@@ -125,6 +126,34 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
         int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode")
+    return out
+
+
+def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+               v_cache: torch.Tensor, block_tables: torch.Tensor,
+               query_start: torch.Tensor, context_lens: torch.Tensor,
+               max_query_len: int, max_context_len: int, sm_scale: float, *,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Chunked causal prefill attention (see pa.h); out [T][Hq][D] fp32."""
+    _need(out, "out", (torch.float32,), 3)
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.float8_e4m3fn, torch.uint8), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_tables, "block_tables", (torch.int32,), 2)
+    _need(query_start, "query_start", (torch.int32,), 1)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    T, Hq, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    S = context_lens.shape[0]
+    if tuple(out.shape) != (T, Hq, D) or Dc != D or query_start.shape[0] != S + 1:
+        raise ValueError("shape mismatch between out, q, caches and query_start")
+    rc = _lib.lib().pa_prefill(
+        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        kv_dtype_of(k_cache), block_tables.data_ptr(), block_tables.shape[1],
+        query_start.data_ptr(), context_lens.data_ptr(), int(max_query_len),
+        int(max_context_len), S, T, Hq, Hkv, D, B, NB, float(sm_scale),
+        _stream_ptr(stream, q.device))
+    _ok(rc, "pa_prefill")
     return out
 
 

@@ -29,6 +29,8 @@ SIGNATURES = {
     "pa_decode_no_alloc": (_i32, [_vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _i32,
                                   _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                   _f32, _i32, _vp]),
+    "pa_prefill": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32,
+                          _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
     "pa_reshape_and_cache": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                     _i32, _i32, _i32, _f32, _f32, _vp]),
     "pa_copy_blocks": (_i32, [_vp, _vp, _vp, _i32, _sz, _i32, _vp]),

@@ -13,6 +13,7 @@
 #include "pa.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 
 namespace {
 
@@ -311,6 +312,73 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   r.max_partitions = static_cast<int>(P);
   return head_dim == 128 ? launch_reduce<128>(r, num_seqs, st, dev)
                          : launch_reduce<64>(r, num_seqs, st, dev);
+}
+
+pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cache,
+                     pa_kv_dtype kv_dtype, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *query_start, const int32_t *context_lens, int max_query_len,
+                     int max_context_len, int num_seqs, int num_tokens, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     float sm_scale, void *stream) {
+  if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq < 0 || max_context_len < 0 || max_query_len < 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  if (kv_dtype != PA_KV_BF16) return PA_ERR_UNSUPPORTED;
+  if (block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PA_ERR_UNSUPPORTED;
+  if (!std::isfinite(sm_scale)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return PA_ERR_INVALID_ARG;
+  const int64_t rows64 = static_cast<int64_t>(num_blocks) * num_kv_heads * pa::kBS;
+  if (rows64 + pa::kBS >= INT32_MAX) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  pa::PrefillParams p{};
+  p.out = out;
+  p.q = static_cast<const uint16_t *>(q);
+  p.block_tables = block_tables;
+  p.query_start = query_start;
+  p.context_lens = context_lens;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.max_context_len = max_context_len;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.tokens_per_tile = pa::kPrefillRows / group;
+  p.num_blocks = num_blocks;
+  p.score_scale = sm_scale * 1.4426950408889634f;
+  const int rows = static_cast<int>(rows64);
+  const int64_t tiles = (static_cast<int64_t>(max_query_len) + p.tokens_per_tile - 1) /
+                        p.tokens_per_tile;
+  if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap tk, tv;
+  const size_t smem = 1024 + 8 * 8192 + 16 * 8 + 16;
+  if (head_dim == 128) {
+    if (!make_cache_tmap<128, false>(&tk, k_cache, rows) ||
+        !make_cache_tmap<128, false>(&tv, v_cache, rows))
+      return PA_ERR_CUDA;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(pa::paged_prefill_kernel<128>, smem, attr_done, dev)) return PA_ERR_CUDA;
+    pa::paged_prefill_kernel<128><<<grid, pa::kDecodeThreads, smem, st>>>(tk, tv, p);
+  } else {
+    if (!make_cache_tmap<64, false>(&tk, k_cache, rows) ||
+        !make_cache_tmap<64, false>(&tv, v_cache, rows))
+      return PA_ERR_CUDA;
+    static std::atomic<uint64_t> attr_done{0};
+    if (!ensure_smem_attr(pa::paged_prefill_kernel<64>, smem, attr_done, dev)) return PA_ERR_CUDA;
+    pa::paged_prefill_kernel<64><<<grid, pa::kDecodeThreads, smem, st>>>(tk, tv, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache,

@@ -72,7 +72,7 @@ WORKLOADS = {
 }
 
 _STREAM_IDS = {"lengths": 1, "q": 2, "k_old": 3, "v_old": 4, "k_new": 5,
-               "v_new": 6, "pool": 7}
+               "v_new": 6, "pool": 7, "q_prefill": 8}
 
 
 def rng(seed: int, workload: str, what: str) -> np.random.Generator:
