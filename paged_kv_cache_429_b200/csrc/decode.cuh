@@ -734,61 +734,92 @@ struct ReduceParams {
   int max_partitions;
 };
 
+// One CTA per (query head, sequence), 8 warps: warp w folds partitions
+// w, w + 8, ... (each lane a D/32-float slice of o_p, several rows in
+// flight), then the warps' partial sums are added in shared memory.
+constexpr int kReduceWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D) paged_decode_reduce_kernel(const ReduceParams p) {
-  extern __shared__ float s_w[];  // [max_partitions] weights
-  __shared__ float s_red[D / 32];
+__global__ void __launch_bounds__(kReduceWarps * 32) paged_decode_reduce_kernel(const ReduceParams p) {
+  constexpr int V = D / 32;  // floats per lane
+  constexpr int U = 4;       // partitions in flight per warp
+  __shared__ float s_acc[kReduceWarps][D];
+  __shared__ float s_l[kReduceWarps];
+  __shared__ float s_m[kReduceWarps];
   const int hq = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   bool bad;
   const int L = clamped_len(p.context_lens, s, p.max_context_len, p.max_blocks_per_seq, &bad);
   const int P = (L + p.partition_tokens - 1) / p.partition_tokens;
   float *out = p.out + (static_cast<int64_t>(s) * p.num_q_heads + hq) * D;
   if (P == 0) {
-    out[tid] = 0.f;
+    if (tid < D) out[tid] = 0.f;
     return;
   }
   const int64_t row0 = (static_cast<int64_t>(s) * p.num_q_heads + hq) * p.max_partitions;
   const float *m = p.ws_m + row0;
   const float *l = p.ws_l + row0;
-  const float *o = p.ws_o + row0 * D;
+  const float *o = p.ws_o + row0 * D + lane * V;
 
   float mx = -INFINITY;
-  for (int i = tid; i < P; i += D) mx = fmaxf(mx, m[i]);
+  for (int i = tid; i < P; i += kReduceWarps * 32) mx = fmaxf(mx, m[i]);
 #pragma unroll
   for (int k = 16; k > 0; k >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
-  if ((tid & 31) == 0) s_red[tid >> 5] = mx;
+  if (lane == 0) s_m[warp] = mx;
   __syncthreads();
-  float M = s_red[0];
+  float M = s_m[0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) M = fmaxf(M, s_red[w]);
-  __syncthreads();
+  for (int w = 1; w < kReduceWarps; ++w) M = fmaxf(M, s_m[w]);
 
-  float sum = 0.f;
-  for (int i = tid; i < P; i += D) {
-    const float w = exp2f(m[i] - M);
-    s_w[i] = w;
-    sum += w * l[i];
+  float acc[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float lsum = 0.f;
+  for (int i0 = warp; i0 < P; i0 += kReduceWarps * U) {
+    float wt[U], row[U][V];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * kReduceWarps;
+      wt[u] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) row[u][v] = 0.f;
+      if (i < P) {
+        wt[u] = exp2f(m[i] - M);
+        lsum += wt[u] * l[i];
+        if constexpr (V == 4) {
+          const float4 x = *reinterpret_cast<const float4 *>(o + static_cast<int64_t>(i) * D);
+          row[u][0] = x.x;
+          row[u][1] = x.y;
+          row[u][2] = x.z;
+          row[u][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2 *>(o + static_cast<int64_t>(i) * D);
+          row[u][0] = x.x;
+          row[u][1] = x.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int v = 0; v < V; ++v) acc[v] += wt[u] * row[u][v];
   }
 #pragma unroll
-  for (int k = 16; k > 0; k >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, k);
-  if ((tid & 31) == 0) s_red[tid >> 5] = sum;
+  for (int v = 0; v < V; ++v) s_acc[warp][lane * V + v] = acc[v];
+  if (lane == 0) s_l[warp] = lsum;
   __syncthreads();
-  float total = 0.f;
+  if (tid < D) {
+    float a = 0.f, t = 0.f;
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) total += s_red[w];
-
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int i = 0;
-  for (; i + 4 <= P; i += 4) {
-    a0 += s_w[i] * o[static_cast<int64_t>(i) * D + tid];
-    a1 += s_w[i + 1] * o[static_cast<int64_t>(i + 1) * D + tid];
-    a2 += s_w[i + 2] * o[static_cast<int64_t>(i + 2) * D + tid];
-    a3 += s_w[i + 3] * o[static_cast<int64_t>(i + 3) * D + tid];
+    for (int w = 0; w < kReduceWarps; ++w) {
+      a += s_acc[w][tid];
+      t += s_l[w];
+    }
+    out[tid] = a / t;
   }
-  for (; i < P; ++i) a0 += s_w[i] * o[static_cast<int64_t>(i) * D + tid];
-  out[tid] = ((a0 + a1) + (a2 + a3)) / total;
 }
 
 }  // namespace pa

@@ -74,6 +74,27 @@ bool make_cache_tmap(CUtensorMap *map, const void *base, int rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Q rows of a prefill tile: a 3-D view [tokens][query heads][head_dim] of
+// the bf16 queries, box (64 dims, the GQA group's heads, tokens of the tile)
+// with the 128-byte swizzle, so a tile lands as 128-byte rows ordered
+// (token, head) — the K-major operand layout of the tensor core.
+bool make_q_tmap(CUtensorMap *map, const void *q, int num_tokens, int num_q_heads,
+                 int head_dim, int group, int tokens_per_tile) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(num_tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group),
+                       static_cast<cuuint32_t>(tokens_per_tile)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename Kern>
 bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int dev) {
   const uint64_t bit = 1ull << (dev & 63);
@@ -103,15 +124,9 @@ pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
 }
 
 template <int D>
-pa_status launch_reduce(const ReduceParams &r, int num_seqs, cudaStream_t stream, int dev) {
-  auto kern = pa::paged_decode_reduce_kernel<D>;
-  const size_t smem = static_cast<size_t>(r.max_partitions) * sizeof(float);
-  static std::atomic<uint64_t> attr_done{0};
-  if (smem > 48 * 1024) {
-    if (!ensure_smem_attr(kern, 227 * 1024, attr_done, dev)) return PA_ERR_CUDA;
-  }
+pa_status launch_reduce(const ReduceParams &r, int num_seqs, cudaStream_t stream) {
   dim3 grid(r.num_q_heads, num_seqs);
-  kern<<<grid, D, smem, stream>>>(r);
+  pa::paged_decode_reduce_kernel<D><<<grid, pa::kReduceWarps * 32, 0, stream>>>(r);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -214,7 +229,7 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
       std::min<int64_t>(max_context_len, static_cast<int64_t>(max_blocks_per_seq) * pa::kBS));
   if (partition_size > 0) {  // forced split: the workspace must fit (host check)
     const int64_t P = (static_cast<int64_t>(ctx_cap) + partition_size - 1) / partition_size;
-    if (P > 65535 || P * 4 > 200 * 1024) return PA_ERR_UNSUPPORTED;
+    if (P > 65535) return PA_ERR_UNSUPPORTED;
     const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap,
                                             partition_size);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
@@ -265,7 +280,7 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   if (psize > 0) {
     P = (static_cast<int64_t>(ctx_cap) + psize - 1) / psize;
     if (P == 0) P = 1;
-    if (P > 65535 || P * 4 > 200 * 1024) return PA_ERR_UNSUPPORTED;
+    if (P > 65535) return PA_ERR_UNSUPPORTED;
     const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap, psize);
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < need)
       return PA_ERR_WORKSPACE;
@@ -310,8 +325,8 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   r.num_q_heads = num_q_heads;
   r.partition_tokens = psize;
   r.max_partitions = static_cast<int>(P);
-  return head_dim == 128 ? launch_reduce<128>(r, num_seqs, st, dev)
-                         : launch_reduce<64>(r, num_seqs, st, dev);
+  return head_dim == 128 ? launch_reduce<128>(r, num_seqs, st)
+                         : launch_reduce<64>(r, num_seqs, st);
 }
 
 pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cache,
@@ -352,7 +367,7 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
   p.group = group;
-  p.tokens_per_tile = pa::kPrefillRows / group;
+  p.tokens_per_tile = pa::kTcRows / group;
   p.num_blocks = num_blocks;
   p.score_scale = sm_scale * 1.4426950408889634f;
   const int rows = static_cast<int>(rows64);
@@ -361,22 +376,27 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  CUtensorMap tk, tv;
-  const size_t smem = 1024 + 8 * 8192 + 16 * 8 + 16;
+  CUtensorMap tq, tk, tv;
+  if (!make_q_tmap(&tq, q, num_tokens, num_q_heads, head_dim, group, p.tokens_per_tile))
+    return PA_ERR_CUDA;
   if (head_dim == 128) {
     if (!make_cache_tmap<128, false>(&tk, k_cache, rows) ||
         !make_cache_tmap<128, false>(&tv, v_cache, rows))
       return PA_ERR_CUDA;
+    auto kern = pa::paged_prefill_kernel<128>;
+    const size_t smem = pa::TcPlan<128>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
-    if (!ensure_smem_attr(pa::paged_prefill_kernel<128>, smem, attr_done, dev)) return PA_ERR_CUDA;
-    pa::paged_prefill_kernel<128><<<grid, pa::kDecodeThreads, smem, st>>>(tk, tv, p);
+    if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
+    kern<<<grid, pa::kTcThreads, smem, st>>>(tq, tk, tv, p);
   } else {
     if (!make_cache_tmap<64, false>(&tk, k_cache, rows) ||
         !make_cache_tmap<64, false>(&tv, v_cache, rows))
       return PA_ERR_CUDA;
+    auto kern = pa::paged_prefill_kernel<64>;
+    const size_t smem = pa::TcPlan<64>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
-    if (!ensure_smem_attr(pa::paged_prefill_kernel<64>, smem, attr_done, dev)) return PA_ERR_CUDA;
-    pa::paged_prefill_kernel<64><<<grid, pa::kDecodeThreads, smem, st>>>(tk, tv, p);
+    if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
+    kern<<<grid, pa::kTcThreads, smem, st>>>(tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -1,4 +1,5 @@
-// Chunked prefill attention over the paged KV cache (bf16), sm_100a.
+// Chunked prefill attention over the paged KV cache (bf16) on the 5th-
+// generation tensor core (tcgen05, tensor memory), sm_100a.
 //
 // "GPU 学习日报 Day 28：vLLM 与 PagedAttention：GPU Memory 管理的艺术" FAQ Q4:
 // prefill KV is written block-wise into the same pool, and chunked prefill
@@ -6,24 +7,47 @@
 // context_lens[s] tokens in the cache; its last n_s tokens are this chunk's
 // queries, and the query at position p attends to keys 0..p.
 //
-// Design: one CTA per (sequence, KV head, tile of query rows); a row is a
-// (token, query head) pair with the head fastest, so the GQA group's heads
-// share every K/V tile. 64 rows per CTA, 16 per consumer warp. A producer
-// warp streams the blocks 0..(block of the tile's last query position)
-// through the same TMA ring as decode; here every stage is read by all four
-// consumer warps (the empty barrier counts four arrivals). Per block, each
-// warp computes S = Q K^T (16 rows x 16 keys, warp MMA with Q fragments
-// kept in registers), the causal mask, an online softmax per row, and
-// O += P V with P taken straight from the score registers (split into high
-// and low bf16 parts) and V through ldmatrix.trans. Key slots past the
-// context end are zeroed in V (they may hold NaN).
+// Design. One CTA per (sequence, KV head, tile of 128 query rows); a row is
+// a (token, query head) pair with the head fastest, so the GQA group's heads
+// share every K/V tile and the rows fill the MMA's M = 128. Keys stream in
+// tiles of 64 (four 16-token blocks). Six warps:
+//   * warp 4 (producer): one 3-D TMA load of the Q rows, then per key tile
+//     the K and V tiles of its four blocks (through the block table) into a
+//     3-stage ring, each stage guarded by full / empty mbarriers.
+//   * warp 5 (MMA): one thread issues tcgen05.mma. S_j = Q K_j^T (M 128,
+//     N 64, fp32 in tensor memory, double-buffered) and O += P_j V_j (N =
+//     head_dim, O in tensor memory), committing to mbarriers: S_j full, P_j's
+//     buffer free, K/V stage free. S_{j+2} is issued right after PV_j, so
+//     the tensor core computes the next scores while the softmax runs.
+//   * warps 0-3 (softmax): thread r owns row r (its tensor-memory lane). It
+//     reads S_j, applies the scale and the causal mask, and keeps a running
+//     max m and sum l in the exp2 domain. The max used for P is only raised
+//     when a row's tile max exceeds it by more than 2^8 (then O's row is
+//     rescaled in tensor memory), so P <= 2^8 and most tiles never touch O.
+//     P is written to shared memory as high and low bf16 parts (~16
+//     significant bits, two MMAs) in the 128-byte-swizzled layout the MMA
+//     reads. Key slots past the context end may hold NaN: their scores are
+//     masked and their V rows zeroed in shared memory before PV reads them.
+//     At the end each thread divides its O row by l and stores it.
+// Shared memory: Q 32 KB, 3 K/V stages of 32 KB, 2 x (P high, P low) of
+// 16 KB (head_dim 128): 193 KB, one CTA per SM. Tensor memory: 256 columns
+// (S0, S1, O). Every wait is bounded; on time-out the kernel flags
+// PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and MMAs and
+// frees its tensor memory.
 #pragma once
 
 #include "decode.cuh"
 
 namespace pa {
 
-constexpr int kPrefillRows = kConsumerWarps * 16;  // query rows per CTA
+constexpr int kTcRows = 128;                    // query rows per CTA (MMA M)
+constexpr int kTcKeys = 64;                     // keys per tile (S MMA N)
+constexpr int kTcBlocks = kTcKeys / kBS;        // blocks per key tile
+constexpr int kTcStages = 3;                    // K/V ring stages
+constexpr int kTcThreads = 6 * 32;              // 4 softmax + producer + MMA
+constexpr int kTcProducerWarp = 4;
+constexpr int kTcMmaWarp = 5;
+constexpr float kTcRescaleLog2 = 8.f;           // raise the max only past 2^8
 
 struct PrefillParams {
   float *out;                   // [T][Hq][D]
@@ -36,30 +60,72 @@ struct PrefillParams {
   int num_q_heads;
   int num_kv_heads;
   int group;
-  int tokens_per_tile;          // query tokens per CTA (64 / group, floor)
+  int tokens_per_tile;          // query tokens per CTA (128 / group, floor)
   int num_blocks;
   float score_scale;            // sm_scale * log2(e)
 };
 
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads)
-    paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                         const __grid_constant__ CUtensorMap tmap_v,
-                         const PrefillParams p) {
-  using G = Geo<D, false>;
-  constexpr int NS = 8;
-  constexpr int KS = D / 16;   // k-steps for S, n-tile pairs for O
-  constexpr int NT = D / 8;    // O n-tiles (8 dims each)
-  constexpr int BPS = G::kBPS;
+struct TcPlan {
+  static constexpr int kHalves = D / 64;                   // 128-byte atoms per row
+  static constexpr int kQHalfBytes = kTcRows * 128;        // [128 rows][64 dims]
+  static constexpr int kQBytes = kHalves * kQHalfBytes;
+  static constexpr int kKVHalfBytes = kTcKeys * 128;       // [64 keys][64 dims]
+  static constexpr int kStageBytes = 2 * kHalves * kKVHalfBytes;  // K halves, V halves
+  static constexpr int kPBytes = kTcRows * 128;            // [128 rows][64 keys] bf16
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kPOff = kStageOff + kTcStages * kStageBytes;
+  static constexpr int kBarOff = kPOff + 4 * kPBytes;      // P: [buffer 2][high, low]
+  // q_full, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int kNumBars = 1 + 2 * kTcStages + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes = 1024 + kBarOff + 8 * kNumBars + 16;
+  static constexpr int kTmemCols = 256;                    // S0 | S1 | O
+  static constexpr int kOCol = 2 * kTcKeys;
+  static_assert(kOCol + D <= kTmemCols, "tensor-memory plan");
+  static_assert(kSmemBytes <= 227 * 1024, "shared-memory plan");
+};
+
+// Bounded wait shared by all roles; on time-out flags the error and the
+// CTA-wide abort word. Returns false if the wait failed or the CTA aborted.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      raise_error(kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                            const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v,
+                            const PrefillParams p) {
+  using TP = TcPlan<D>;
+  constexpr int H = TP::kHalves;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
-  const uint32_t ring = (raw_u32 + 1023u) & ~1023u;
-  uint8_t *base_ptr = smem_raw + (ring - raw_u32);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(base_ptr + NS * G::kStageBytes);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8u * NS;
-  volatile int *s_abort = reinterpret_cast<volatile int *>(bars + 2 * NS);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+  uint8_t *base_ptr = smem_raw + (base - raw_u32);
+  const uint32_t sq = base;                        // Q half x at sq + x * kQHalfBytes
+  const uint32_t sring = base + TP::kStageOff;     // stage st at sring + st * kStageBytes
+  const uint32_t sp = base + TP::kPOff;            // P buffer b: high at sp + 2b kPBytes
+  const uint32_t bar_q = base + TP::kBarOff;
+  const uint32_t bar_kv_full = bar_q + 8;
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * kTcStages;
+  const uint32_t bar_s_full = bar_kv_empty + 8 * kTcStages;
+  const uint32_t bar_p_full = bar_s_full + 16;
+  const uint32_t bar_pv_done = bar_p_full + 16;
+  const uint32_t bar_drain = bar_pv_done + 16;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base_ptr + TP::kBarOff + 8 * TP::kNumBars);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int qt = blockIdx.x;
   const int h = blockIdx.y;
@@ -71,257 +137,289 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int L = clamped_len(p.context_lens, s, p.max_context_len, p.max_blocks_per_seq, &bad_len);
   const int q0 = p.query_start[s];
   const int n = min(p.query_start[s + 1] - q0, L);  // chunk length
-  const int t0 = qt * p.tokens_per_tile;            // first chunk token of this tile
+  const int tpt = p.tokens_per_tile;
+  const int t0 = qt * tpt;                          // first chunk token of this tile
   if (t0 >= n) return;
   if (bad_len && threadIdx.x == 0 && qt == 0) raise_error(kErrContextClamp);
-  const int t1 = min(n, t0 + p.tokens_per_tile);    // one past the last
-  const int last_pos = L - n + t1 - 1;              // largest query position here
-  const int nblk = last_pos / kBS + 1;              // blocks 0..nblk-1 are needed
-  const int nst = (nblk + BPS - 1) / BPS;
+  const int group = p.group;
+  const int t1 = min(n, t0 + tpt);
+  const int ctx0 = L - n;                           // position of chunk token 0
+  const int kmax = ctx0 + t1 - 1;                   // last key any row here sees
+  const int nblk = kmax / kBS + 1;
+  const int ntiles = kmax / kTcKeys + 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(full0 + 8u * i, 1);
-      mbar_init(empty0 + 8u * i, kConsumerWarps);
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(bar_kv_full + 8u * i, 1);
+      mbar_init(bar_kv_empty + 8u * i, 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s_full + 8u * i, 1);
+      mbar_init(bar_p_full + 8u * i, 4 * 32);
+      mbar_init(bar_pv_done + 8u * i, 1);
+    }
+    mbar_init(bar_drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
+  if (warp == kTcMmaWarp) {
+    tmem_alloc(smem_u32(s_tmem), TP::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
   __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *s_tmem;
 
-  if (warp == kConsumerWarps) {
-    // ---------------------------------------------------------- producer
+  if (warp == kTcProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      mbar_arrive_expect_tx(bar_q, H * 128 * group * tpt);
+#pragma unroll
+      for (int x = 0; x < H; ++x)
+        tma_load_3d(sq + x * TP::kQHalfBytes, &tmap_q, bar_q, 64 * x, h * group, q0 + t0);
+    }
     const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
     const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
-    int issued = 0;
     bool ok = true, bad_id = false;
-    for (int jb = 0; jb < nst * BPS && ok; jb += 32) {
-      const int mine = (jb + lane < nblk) ? bt[jb + lane] : -1;
-      const int i_end = min(nst, (jb + 32) / BPS);
-      for (int i = jb / BPS; i < i_end; ++i) {
-        int phys[BPS];
-#pragma unroll
-        for (int b = 0; b < BPS; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, i * BPS + b - jb);
-        if (lane == 0) {
-          const int st = i % NS;
-          if (i >= NS && !mbar_try_wait(empty0 + 8u * st, ((i / NS) - 1) & 1)) {
-            if (*s_abort) {
-              ok = false;
-            } else if (!mbar_wait_bounded(empty0 + 8u * st, ((i / NS) - 1) & 1, kWaitLimitNs)) {
-              ok = false;
-              *s_abort = 1;
-              raise_error(kErrWaitTimeout);
-            }
-          }
-          if (ok) {
-            const uint32_t fb = full0 + 8u * st;
-            const uint32_t kdst = ring + st * G::kStageBytes;
-            const uint32_t vdst = kdst + BPS * G::kTileBytes;
-            mbar_arrive_expect_tx(fb, G::kStageBytes);
-#pragma unroll
-            for (int b = 0; b < BPS; ++b) {
-              const bool real = i * BPS + b < nblk;
-              int y;
-              if (!real || phys[b] < 0 || phys[b] >= p.num_blocks) {
-                y = total_rows;
-                bad_id |= real;
-              } else {
-                y = (phys[b] * p.num_kv_heads + h) * kBS;
-              }
-#pragma unroll
-              for (int x = 0; x < G::kBoxes; ++x) {
-                tma_load_2d(kdst + b * G::kTileBytes + x * G::kBoxBytes, &tmap_k, fb,
-                            x * (G::kBoxRow / G::kEB), y);
-                tma_load_2d(vdst + b * G::kTileBytes + x * G::kBoxBytes, &tmap_v, fb,
-                            x * (G::kBoxRow / G::kEB), y);
-              }
-            }
-            issued = i + 1;
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+    int issued = 0;
+    int mine = -1;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      // 32 table entries (8 tiles) per warp load
+      if ((j & 7) == 0) {
+        const int jb = j * kTcBlocks + lane;
+        mine = jb < nblk ? bt[jb] : -1;
       }
+      int phys[kTcBlocks];
+#pragma unroll
+      for (int b = 0; b < kTcBlocks; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, (j & 7) * kTcBlocks + b);
+      if (lane == 0) {
+        const int st = j % kTcStages;
+        if (j >= kTcStages) ok = tc_wait(bar_kv_empty + 8u * st, ((j / kTcStages) - 1) & 1, s_abort);
+        if (ok) {
+          const uint32_t full = bar_kv_full + 8u * st;
+          const uint32_t kst = sring + st * TP::kStageBytes;
+          mbar_arrive_expect_tx(full, TP::kStageBytes);
+#pragma unroll
+          for (int b = 0; b < kTcBlocks; ++b) {
+            const bool real = j * kTcBlocks + b < nblk;
+            int y;
+            if (!real || phys[b] < 0 || phys[b] >= p.num_blocks) {
+              y = total_rows;  // past the tensor's end: TMA fills zeros
+              bad_id |= real;
+            } else {
+              y = (phys[b] * p.num_kv_heads + h) * kBS;
+            }
+#pragma unroll
+            for (int x = 0; x < H; ++x) {
+              tma_load_2d(kst + x * TP::kKVHalfBytes + b * 2048, &tmap_k, full, 64 * x, y);
+              tma_load_2d(kst + (H + x) * TP::kKVHalfBytes + b * 2048, &tmap_v, full, 64 * x, y);
+            }
+          }
+          issued = j + 1;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (lane == 0) {
       if (bad_id) raise_error(kErrBlockRange);
-      for (int i = max(0, issued - NS); i < issued; ++i)
-        mbar_wait_bounded(full0 + 8u * (i % NS), (i / NS) & 1, kWaitLimitNs);
+      // no bulk copy may still be landing when the CTA exits
+      mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
+      for (int j = max(0, issued - kTcStages); j < issued; ++j)
+        mbar_wait_bounded(bar_kv_full + 8u * (j % kTcStages), (j / kTcStages) & 1, kWaitLimitNs);
     }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int gq = lane >> 2;
-  const int qd = lane & 3;
-  const int mi = lane >> 3;
-  const int mrow = lane & 7;
-  const int group = p.group;
-  // this thread's two rows: gq and gq + 8 of the warp's 16
-  int qpos[2];       // query position (causal bound); -1 never happens
-  bool live[2];
-  const uint16_t *qrow[2];
-  int orow[2], ohead[2];
+  } else if (warp == kTcMmaWarp) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t id_s = tc_idesc_bf16(kTcRows, kTcKeys, false);
+      constexpr uint32_t id_pv = tc_idesc_bf16(kTcRows, D, true);
+      bool ok = tc_wait(bar_q, 0, s_abort);
+      // S_j = Q K_j^T into S buffer j % 2
+      auto issue_s = [&](int j) {
+        const int st = j % kTcStages;
+        ok = tc_wait(bar_kv_full + 8u * st, (j / kTcStages) & 1, s_abort);
+        if (!ok) return;
+        tc_fence_after_sync();
+        const uint32_t kst = sring + st * TP::kStageBytes;
+        const uint32_t d = tmem + (j & 1) * kTcKeys;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int R = warp * 16 + gq + 8 * r;  // row in the CTA tile
-    const int ti = R / group;               // token in the tile
-    const int hn = R - ti * group;           // head within the group
-    const int tok = t0 + ti;
-    live[r] = ti < p.tokens_per_tile && tok < t1;
-    qpos[r] = live[r] ? L - n + tok : L - 1;  // a dead row sees all keys (q = 0)
-    orow[r] = q0 + tok;
-    ohead[r] = h * group + hn;
-    qrow[r] = p.q + (static_cast<int64_t>(orow[r]) * p.num_q_heads + ohead[r]) * D;
-  }
-  // Q as the A operand: a0/a2 = row gq, a1/a3 = row gq+8; k-slots 2qd(+8)
-  uint32_t qa[KS][4];
-#pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    qa[ks][0] = live[0] ? *reinterpret_cast<const uint32_t *>(qrow[0] + 16 * ks + 2 * qd) : 0u;
-    qa[ks][1] = live[1] ? *reinterpret_cast<const uint32_t *>(qrow[1] + 16 * ks + 2 * qd) : 0u;
-    qa[ks][2] = live[0] ? *reinterpret_cast<const uint32_t *>(qrow[0] + 16 * ks + 8 + 2 * qd) : 0u;
-    qa[ks][3] = live[1] ? *reinterpret_cast<const uint32_t *>(qrow[1] + 16 * ks + 8 + 2 * qd) : 0u;
-  }
-  float o[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  const int warp_last = max(qpos[0], qpos[1]);  // per-thread; warp max below
-  int wmax = warp_last;
-#pragma unroll
-  for (int o2 = 1; o2 < 32; o2 <<= 1) wmax = max(wmax, __shfl_xor_sync(0xffffffffu, wmax, o2));
-
-  bool aborted = false;
-  for (int i = 0; i < nst; ++i) {
-    const int st = i % NS;
-    if (!aborted) {
-      const bool got = mbar_wait_bounded(full0 + 8u * st, (i / NS) & 1, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, got)) {
-        aborted = true;
-        if (lane == 0) {
-          *s_abort = 1;
-          raise_error(kErrWaitTimeout);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;  // 16 dims = 32 bytes of the atom row
+          const uint64_t a = tc_desc_sw128(sq + (ks >> 2) * TP::kQHalfBytes + off, 16, 1024);
+          const uint64_t b = tc_desc_sw128(kst + (ks >> 2) * TP::kKVHalfBytes + off, 16, 1024);
+          tc_mma_ss(d, a, b, id_s, ks > 0);
         }
+        tc_commit(bar_s_full + 8u * (j & 1));
+      };
+      if (ok) issue_s(0);
+      if (ok && ntiles > 1) issue_s(1);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        ok = tc_wait(bar_p_full + 8u * (j & 1), (j >> 1) & 1, s_abort);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const int st = j % kTcStages;
+        const uint32_t vst = sring + st * TP::kStageBytes + H * TP::kKVHalfBytes;
+        const uint32_t pb = sp + (j & 1) * 2 * TP::kPBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBlocks; ++kk) {
+          // V: 16 keys (two 8-key atoms, 1024 B apart) x head_dim (64-dim
+          // atoms kKVHalfBytes apart), dims contiguous
+          const uint64_t b = tc_desc_sw128(vst + kk * 2048, TP::kKVHalfBytes, 1024);
+          const uint64_t a_hi = tc_desc_sw128(pb + kk * 32, 16, 1024);
+          const uint64_t a_lo = tc_desc_sw128(pb + TP::kPBytes + kk * 32, 16, 1024);
+          tc_mma_ss(tmem + TP::kOCol, a_hi, b, id_pv, j > 0 || kk > 0);
+          tc_mma_ss(tmem + TP::kOCol, a_lo, b, id_pv, true);
+        }
+        tc_commit(bar_pv_done + 8u * (j & 1));
+        tc_commit(bar_kv_empty + 8u * st);
+        if (j + 2 < ntiles) issue_s(j + 2);
       }
-    }
-    if (!aborted) {
-#pragma unroll
-      for (int b = 0; b < BPS; ++b) {
-        const int j = i * BPS + b;  // block index = first key position / 16
-        if (j >= nblk || j * kBS > wmax) continue;  // no key here for this warp
-        const uint32_t kt = ring + st * G::kStageBytes + b * G::kTileBytes;
-        const uint32_t vt = ring + st * G::kStageBytes + (BPS + b) * G::kTileBytes;
-        // ---- S = Q K^T: two n-tiles of 8 keys
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t b00, b01, b10, b11;  // (keys 0-7 | 8-15) x (dims lo | hi)
-          ldsm_x4(kt + swz<D, false>((mi >> 1) * 8 + mrow, 32 * ks + (mi & 1) * 16), b00, b01,
-                  b10, b11);
-          mma_16816<false>(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-          mma_16816<false>(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
-        }
-        // ---- causal mask and online softmax per row
-        float z[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = j * kBS + nt * 8 + 2 * qd + (e & 1);
-            const int r = e >> 1;
-            z[nt][e] = (key <= qpos[r]) ? sc[nt][e] * p.score_scale : -INFINITY;
-          }
-        float alpha[2];
-        bool rescale = false;
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          float mx = fmaxf(fmaxf(z[0][2 * r], z[0][2 * r + 1]), fmaxf(z[1][2 * r], z[1][2 * r + 1]));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float mn = fmaxf(m_run[r], mx);
-          // a row with no visible key yet keeps m = -inf: exp2 of -inf - -inf is avoided
-          alpha[r] = (mn == -INFINITY) ? 1.f : exp2f(m_run[r] - mn);
-          rescale |= (mn != m_run[r]);
-          m_run[r] = mn;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float &zz = z[nt][2 * r + c];
-              zz = (mn == -INFINITY) ? 0.f : exp2f(zz - mn);
-            }
-          l_run[r] = l_run[r] * alpha[r] + (z[0][2 * r] + z[0][2 * r + 1] + z[1][2 * r] + z[1][2 * r + 1]);
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            o[nt][0] *= alpha[0];
-            o[nt][1] *= alpha[0];
-            o[nt][2] *= alpha[1];
-            o[nt][3] *= alpha[1];
-          }
-        }
-        // ---- P as the A operand (keys are the k dimension): hi and lo parts
-        uint32_t ph[4], pl[4];
-        {
-          const uint32_t h0 = pack2<false>(z[0][0], z[0][1]), h1 = pack2<false>(z[0][2], z[0][3]);
-          const uint32_t h2 = pack2<false>(z[1][0], z[1][1]), h3 = pack2<false>(z[1][2], z[1][3]);
-          float u[8];
-          unpack2<false>(h0, u[0], u[1]);
-          unpack2<false>(h1, u[2], u[3]);
-          unpack2<false>(h2, u[4], u[5]);
-          unpack2<false>(h3, u[6], u[7]);
-          ph[0] = h0;
-          ph[1] = h1;
-          ph[2] = h2;
-          ph[3] = h3;
-          pl[0] = pack2<false>(z[0][0] - u[0], z[0][1] - u[1]);
-          pl[1] = pack2<false>(z[0][2] - u[2], z[0][3] - u[3]);
-          pl[2] = pack2<false>(z[1][0] - u[4], z[1][1] - u[5]);
-          pl[3] = pack2<false>(z[1][2] - u[6], z[1][3] - u[7]);
-        }
-        // key slots past the context end may hold NaN: zero their V
-        const int vb = L - j * kBS;  // real keys in this block
-        uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;
-        if (vb < kBS) {
-          m0 = (2 * qd < vb ? 0x0000ffffu : 0u) | (2 * qd + 1 < vb ? 0xffff0000u : 0u);
-          m1 = (2 * qd + 8 < vb ? 0x0000ffffu : 0u) | (2 * qd + 9 < vb ? 0xffff0000u : 0u);
-        }
-        // ---- O += P V: V^T fragments via ldmatrix.trans, two n-tiles per load
-#pragma unroll
-        for (int np = 0; np < KS; ++np) {
-          uint32_t v0, v1, v2, v3;  // (keys 0-7 | 8-15) x (dims 16np..+7 | +8..+15)
-          ldsm_x4_trans(vt + swz<D, false>((mi & 1) * 8 + mrow, 32 * np + (mi >> 1) * 16), v0, v1,
-                        v2, v3);
-          v0 &= m0;
-          v1 &= m1;
-          v2 &= m0;
-          v3 &= m1;
-          mma_16816<false>(o[2 * np], ph[0], ph[1], ph[2], ph[3], v0, v1);
-          mma_16816<false>(o[2 * np], pl[0], pl[1], pl[2], pl[3], v0, v1);
-          mma_16816<false>(o[2 * np + 1], ph[0], ph[1], ph[2], ph[3], v2, v3);
-          mma_16816<false>(o[2 * np + 1], pl[0], pl[1], pl[2], pl[3], v2, v3);
-        }
-      }
+      // every MMA issued here has completed before tensor memory is freed
+      tc_commit(bar_drain);
+      mbar_wait_bounded(bar_drain, 0, kWaitLimitNs);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8u * st);
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int r = warp * 32 + lane;               // row = tensor-memory lane
+    const int t = r / group;
+    const int nh = r - t * group;
+    const bool valid = t < tpt && t0 + t < n;
+    const int klim = valid ? ctx0 + t0 + t : -1;  // keys <= klim are visible
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    // the tile holding the context's last, partly filled block: zero the V
+    // rows past the context end (NaN allowed there) before PV reads them
+    const int tail = L % kBS;
+    const int zero_tile = (tail != 0 && (L - 1) / kBS < nblk) ? (L - 1) / kTcKeys : -1;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8u * (j & 1), (j >> 1) & 1, s_abort));
+      if (!ok) break;
+      tc_fence_after_sync();
+      uint32_t sr[2][32];
+      tc_ld_32x32b_x32(trow + (j & 1) * kTcKeys, sr[0]);
+      tc_ld_32x32b_x32(trow + (j & 1) * kTcKeys + 32, sr[1]);
+      tc_wait_ld();
+      float z[kTcKeys];
+      float mt = -INFINITY;
+      const int kb = j * kTcKeys;
+      if (kb + kTcKeys - 1 > klim) {
+#pragma unroll
+        for (int c = 0; c < kTcKeys; ++c) {
+          const float v = __uint_as_float(sr[c >> 5][c & 31]) * p.score_scale;
+          z[c] = (kb + c > klim) ? -INFINITY : v;
+          mt = fmaxf(mt, z[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kTcKeys; ++c) {
+          z[c] = __uint_as_float(sr[c >> 5][c & 31]) * p.score_scale;
+          mt = fmaxf(mt, z[c]);
+        }
+      }
+      const float m_new = (mt > m_used + kTcRescaleLog2) ? mt : m_used;
+      const bool raise = m_new != m_used;
+      const float alpha = raise ? exp2f(m_used - m_new) : 1.f;
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        // O must hold PV_{j-1} before its rows are rescaled
+        ok = __all_sync(0xffffffffu,
+                        tc_wait(bar_pv_done + 8u * ((j - 1) & 1), ((j - 1) >> 1) & 1, s_abort));
+        if (!ok) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tc_ld_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tc_st_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+        }
+        tc_wait_st();
+      }
+      l *= alpha;
+      m_used = m_new;
+      // P buffer j % 2 is free once PV_{j-2} has completed
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu,
+                        tc_wait(bar_pv_done + 8u * (j & 1), ((j - 2) >> 1) & 1, s_abort));
+        if (!ok) break;
+      }
+      const uint32_t phi = sp + (j & 1) * 2 * TP::kPBytes + r * 128;
+      const uint32_t plo = phi + TP::kPBytes;
+      const bool live = valid && m_used != -INFINITY;
+      float rs = 0.f;
+#pragma unroll
+      for (int q = 0; q < kTcKeys / 8; ++q) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = q * 8 + 2 * e;
+          const float p0 = live ? exp2f(z[c] - m_used) : 0.f;
+          const float p1 = live ? exp2f(z[c + 1] - m_used) : 0.f;
+          rs += p0 + p1;
+          hi[e] = pack2<false>(p0, p1);
+          float u0, u1;
+          unpack2<false>(hi[e], u0, u1);
+          lo[e] = pack2<false>(p0 - u0, p1 - u1);
+        }
+        const uint32_t chunk = static_cast<uint32_t>((q ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(phi + chunk), "r"(hi[0]),
+                     "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
+                     : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(plo + chunk), "r"(lo[0]),
+                     "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
+                     : "memory");
+      }
+      l += rs;
+      if (j == zero_tile && warp == 0) {
+        const uint32_t vb = sring + (j % kTcStages) * TP::kStageBytes + H * TP::kKVHalfBytes +
+                            (((L - 1) / kBS) % kTcBlocks) * 2048;
+        const int nrow = kBS - tail;
+        for (int i = lane; i < nrow * 8 * H; i += 32) {
+          const int row = tail + i / (8 * H);
+          const int rem = i % (8 * H);
+          const uint32_t a = vb + (rem >> 3) * TP::kKVHalfBytes + row * 128 + (rem & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive(bar_p_full + 8u * (j & 1));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok)
+      ok = __all_sync(0xffffffffu, tc_wait(bar_pv_done + 8u * ((ntiles - 1) & 1),
+                                           ((ntiles - 1) >> 1) & 1, s_abort));
+    if (ok) {
+      tc_fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float *orow = p.out + (static_cast<int64_t>(q0 + t0 + t) * p.num_q_heads + h * group + nh) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tc_ld_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4 *>(orow + cc * 32 + e) =
+                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        }
+      }
+    }
+    tc_fence_before_sync();
   }
-
-  // ---- normalise and write this thread's rows
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float l = l_run[r];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if (!live[r]) continue;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    float *dst = p.out + (static_cast<int64_t>(orow[r]) * p.num_q_heads + ohead[r]) * D;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      *reinterpret_cast<float2 *>(dst + 8 * nt + 2 * qd) =
-          make_float2(o[nt][2 * r] * inv, o[nt][2 * r + 1] * inv);
+  __syncthreads();
+  if (warp == kTcMmaWarp) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TP::kTmemCols);
   }
 }
 

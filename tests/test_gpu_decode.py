@@ -100,6 +100,25 @@ def test_edge_lengths_heads_dtypes(D, fp8, hq, hkv):
     check_batch(b, paths=(0, 16, 512, -1))
 
 
+SPLIT_EDGE_LENS = [1, 2, 15, 16, 17, 511, 512, 513, 1024, 1025, 2047, 2048, 2049, 2560, 3000,
+                   3072]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("hq,hkv", [(16, 4), (64, 4)])
+def test_split_chunks_of_several_partitions(D, fp8, hq, hkv):
+    """160 sequences x 4 KV heads: enough CTAs that the split path streams
+    chunks of several 512-token partitions per CTA (merged after each). The
+    lengths cover one-token and partial last partitions and chunk
+    boundaries (2048 / 2049 tokens for 4-partition chunks)."""
+    rest = np.random.default_rng(11).integers(1, 3073, size=160 - len(SPLIT_EDGE_LENS))
+    lens = np.concatenate([SPLIT_EDGE_LENS, rest])
+    w = synth.Workload(f"owned{D}{int(fp8)}{hq}", len(lens), hq, hkv, D, fp8)
+    b = DecodeBatch.build(w, 7, lens=lens)
+    check_batch(b, subset=list(range(len(SPLIT_EDGE_LENS))) + [100, 159], paths=(512, 0))
+
+
 def test_single_and_split_agree_closely():
     b = DecodeBatch.build(synth.WORKLOADS["tiny"], 4)
     b.step(partition_size=0)
