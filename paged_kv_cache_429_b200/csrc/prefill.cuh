@@ -91,7 +91,7 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -306,25 +306,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_ld_32x32b_x32(trow + (j & 1) * kTcKeys + 32, sr[1]);
       tc_wait_ld();
       float z[kTcKeys];
-      float mt = -INFINITY;
       const int kb = j * kTcKeys;
+#pragma unroll
+      for (int c = 0; c < kTcKeys; ++c) z[c] = __uint_as_float(sr[c >> 5][c & 31]) * p.score_scale;
       if (kb + kTcKeys - 1 > klim) {
 #pragma unroll
-        for (int c = 0; c < kTcKeys; ++c) {
-          const float v = __uint_as_float(sr[c >> 5][c & 31]) * p.score_scale;
-          z[c] = (kb + c > klim) ? -INFINITY : v;
-          mt = fmaxf(mt, z[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kTcKeys; ++c) {
-          z[c] = __uint_as_float(sr[c >> 5][c & 31]) * p.score_scale;
-          mt = fmaxf(mt, z[c]);
-        }
+        for (int c = 0; c < kTcKeys; ++c)
+          if (kb + c > klim) z[c] = -INFINITY;
       }
+      // tile max as a tree (independent chains)
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(z[i], z[i + 8]);
+#pragma unroll
+      for (int c = 16; c < kTcKeys; c += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[c + i]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = (mt > m_used + kTcRescaleLog2) ? mt : m_used;
       const bool raise = m_new != m_used;
-      const float alpha = raise ? exp2f(m_used - m_new) : 1.f;
+      const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
         // O must hold PV_{j-1} before its rows are rescaled
         ok = __all_sync(0xffffffffu,
@@ -353,16 +355,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t phi = sp + (j & 1) * 2 * TP::kPBytes + r * 128;
       const uint32_t plo = phi + TP::kPBytes;
       const bool live = valid && m_used != -INFINITY;
-      float rs = 0.f;
+      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < kTcKeys / 8; ++q) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = q * 8 + 2 * e;
-          const float p0 = live ? exp2f(z[c] - m_used) : 0.f;
-          const float p1 = live ? exp2f(z[c + 1] - m_used) : 0.f;
-          rs += p0 + p1;
+          const float p0 = live ? ex2_approx(z[c] - m_used) : 0.f;
+          const float p1 = live ? ex2_approx(z[c + 1] - m_used) : 0.f;
+          rsum[e] += p0 + p1;
           hi[e] = pack2<false>(p0, p1);
           float u0, u1;
           unpack2<false>(hi[e], u0, u1);
@@ -376,6 +378,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
                      : "memory");
       }
+      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       l += rs;
       if (j == zero_tile && warp == 0) {
         const uint32_t vb = sring + (j % kTcStages) * TP::kStageBytes + H * TP::kKVHalfBytes +
