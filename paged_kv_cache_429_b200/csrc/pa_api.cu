@@ -371,8 +371,8 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   p.num_blocks = num_blocks;
   p.score_scale = sm_scale * 1.4426950408889634f;
   const int rows = static_cast<int>(rows64);
-  const int64_t tiles = (static_cast<int64_t>(max_query_len) + p.tokens_per_tile - 1) /
-                        p.tokens_per_tile;
+  const int64_t cta_tokens = static_cast<int64_t>(pa::kTcQTiles) * p.tokens_per_tile;
+  const int64_t tiles = (static_cast<int64_t>(max_query_len) + cta_tokens - 1) / cta_tokens;
   if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

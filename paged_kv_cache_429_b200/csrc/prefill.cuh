@@ -7,46 +7,58 @@
 // context_lens[s] tokens in the cache; its last n_s tokens are this chunk's
 // queries, and the query at position p attends to keys 0..p.
 //
-// Design. One CTA per (sequence, KV head, tile of 128 query rows); a row is
-// a (token, query head) pair with the head fastest, so the GQA group's heads
-// share every K/V tile and the rows fill the MMA's M = 128. Keys stream in
-// tiles of 64 (four 16-token blocks). Six warps:
-//   * warp 4 (producer): one 3-D TMA load of the Q rows, then per key tile
-//     the K and V tiles of its four blocks (through the block table) into a
-//     3-stage ring, each stage guarded by full / empty mbarriers.
-//   * warp 5 (MMA): one thread issues tcgen05.mma. S_j = Q K_j^T (M 128,
-//     N 64, fp32 in tensor memory, double-buffered) and O += P_j V_j (N =
-//     head_dim, O in tensor memory), committing to mbarriers: S_j full, P_j's
-//     buffer free, K/V stage free. S_{j+2} is issued right after PV_j, so
-//     the tensor core computes the next scores while the softmax runs.
-//   * warps 0-3 (softmax): thread r owns row r (its tensor-memory lane). It
-//     reads S_j, applies the scale and the causal mask, and keeps a running
-//     max m and sum l in the exp2 domain. The max used for P is only raised
-//     when a row's tile max exceeds it by more than 2^8 (then O's row is
-//     rescaled in tensor memory), so P <= 2^8 and most tiles never touch O.
-//     P is written to shared memory as high and low bf16 parts (~16
-//     significant bits, two MMAs) in the 128-byte-swizzled layout the MMA
-//     reads. Key slots past the context end may hold NaN: their scores are
-//     masked and their V rows zeroed in shared memory before PV reads them.
-//     At the end each thread divides its O row by l and stores it.
-// Shared memory: Q 32 KB, 3 K/V stages of 32 KB, 2 x (P high, P low) of
-// 16 KB (head_dim 128): 193 KB, one CTA per SM. Tensor memory: 256 columns
-// (S0, S1, O). Every wait is bounded; on time-out the kernel flags
-// PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and MMAs and
-// frees its tensor memory.
+// Design. One CTA per (sequence, KV head, two tiles of 128 query rows); a
+// row is a (token, query head) pair with the head fastest, so the GQA
+// group's heads share every K/V tile and a tile fills the MMA's M = 128.
+// Both query tiles consume every K/V tile the CTA streams, so each K/V byte
+// feeds 256 rows. Keys stream in tiles of 64 (four 16-token blocks). Eleven
+// warps:
+//   * warps 8 and 9 (producers): 3-D TMA loads of the two tiles' Q rows,
+//     then per key tile the K (warp 8) and V (warp 9) tiles of its four
+//     blocks (through the block table) into a 4-stage K ring, freed once
+//     both tiles' S_j are computed, and a 3-stage V ring, freed after both
+//     PV_j; every stage is guarded by full / empty mbarriers.
+//   * warp 10 (MMA): one thread issues tcgen05.mma: per query tile g,
+//     S_gj = Q_g K_j^T (M 128, N 64, fp32) into one of two tensor-memory S
+//     buffers of that tile, and O_g += P_gj V_j (N = head_dim) into the
+//     tile's O, committing to mbarriers: S full, K stage free, PV done, V
+//     stage free. S_g(j+2) reuses S_gj's buffer and is issued right after
+//     PV_j (one thread's MMAs run in issue order), so the next scores are
+//     computed while the softmax runs.
+//   * warps 0-3 / 4-7 (softmax of query tile 0 / 1): thread (warp w) owns
+//     row 32 (w % 4) + lane of its tile (its tensor-memory lane). It reads
+//     S, applies the scale and the causal mask, and keeps a running max m
+//     and sum l in the exp2 domain. The max used for P is only raised when
+//     a row's tile max exceeds it by more than 2^8 (then O's row is
+//     rescaled in tensor memory), so P <= 2^8 and most key tiles never
+//     touch O. P is written back into S's tensor-memory columns as high
+//     and low bf16 parts (~16 significant bits, two MMAs), and PV takes A
+//     from there, so the PV MMAs read only V from shared memory. Key slots
+//     past the context end may hold NaN: their scores are masked and their
+//     V rows zeroed in shared memory before PV reads them. At the end each
+//     thread divides its O row by l and stores it.
+// Shared memory: Q 64 KB, 4 K and 3 V stages of 16 KB (head_dim 128):
+// 176 KB, one CTA per SM. Tensor memory: all 512 columns (2 x 2 S buffers
+// of 64, 2 O of head_dim). Every wait is bounded; on time-out the kernel
+// flags PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and
+// MMAs and frees its tensor memory.
 #pragma once
 
 #include "decode.cuh"
 
 namespace pa {
 
-constexpr int kTcRows = 128;                    // query rows per CTA (MMA M)
+constexpr int kTcRows = 128;                    // rows per query tile (MMA M)
+constexpr int kTcQTiles = 2;                    // query tiles per CTA
 constexpr int kTcKeys = 64;                     // keys per tile (S MMA N)
 constexpr int kTcBlocks = kTcKeys / kBS;        // blocks per key tile
-constexpr int kTcStages = 3;                    // K/V ring stages
-constexpr int kTcThreads = 6 * 32;              // 4 softmax + producer + MMA
-constexpr int kTcProducerWarp = 4;
-constexpr int kTcMmaWarp = 5;
+constexpr int kTcKStages = 4;                   // K ring stages (freed after S)
+constexpr int kTcVStages = 3;                   // V ring stages (freed after PV)
+constexpr int kTcSoftmaxWarps = 4 * kTcQTiles;  // one warpgroup per query tile
+constexpr int kTcThreads = (kTcSoftmaxWarps + 3) * 32;  // + 2 producers + MMA
+constexpr int kTcKWarp = kTcSoftmaxWarps;       // Q and K loads
+constexpr int kTcVWarp = kTcSoftmaxWarps + 1;   // V loads
+constexpr int kTcMmaWarp = kTcSoftmaxWarps + 2;
 constexpr float kTcRescaleLog2 = 8.f;           // raise the max only past 2^8
 
 struct PrefillParams {
@@ -60,7 +72,7 @@ struct PrefillParams {
   int num_q_heads;
   int num_kv_heads;
   int group;
-  int tokens_per_tile;          // query tokens per CTA (128 / group, floor)
+  int tokens_per_tile;          // query tokens per 128-row tile (128 / group, floor)
   int num_blocks;
   float score_scale;            // sm_scale * log2(e)
 };
@@ -69,19 +81,19 @@ template <int D>
 struct TcPlan {
   static constexpr int kHalves = D / 64;                   // 128-byte atoms per row
   static constexpr int kQHalfBytes = kTcRows * 128;        // [128 rows][64 dims]
-  static constexpr int kQBytes = kHalves * kQHalfBytes;
+  static constexpr int kQBytes = kHalves * kQHalfBytes;    // one query tile
   static constexpr int kKVHalfBytes = kTcKeys * 128;       // [64 keys][64 dims]
-  static constexpr int kStageBytes = 2 * kHalves * kKVHalfBytes;  // K halves, V halves
-  static constexpr int kPBytes = kTcRows * 128;            // [128 rows][64 keys] bf16
-  static constexpr int kStageOff = kQBytes;
-  static constexpr int kPOff = kStageOff + kTcStages * kStageBytes;
-  static constexpr int kBarOff = kPOff + 4 * kPBytes;      // P: [buffer 2][high, low]
-  // q_full, kv_full[3], kv_empty[3], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kTcStages + 2 + 2 + 2 + 1;
+  static constexpr int kTileBytes = kHalves * kKVHalfBytes;  // one K (or V) tile
+  static constexpr int kKOff = kTcQTiles * kQBytes;
+  static constexpr int kVOff = kKOff + kTcKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kTcVStages * kTileBytes;
+  // q_full, k_full[4], k_empty[4], v_full[3], v_empty[3], and per query
+  // tile s_full[2], p_full[2], pv_done[2]; drain
+  static constexpr int kNumBars = 1 + 2 * kTcKStages + 2 * kTcVStages + 6 * kTcQTiles + 1;
   static constexpr int kSmemBytes = 1024 + kBarOff + 8 * kNumBars + 16;
-  static constexpr int kTmemCols = 256;                    // S0 | S1 | O
-  static constexpr int kOCol = 2 * kTcKeys;
-  static_assert(kOCol + D <= kTmemCols, "tensor-memory plan");
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol = 2 * kTcQTiles * kTcKeys;    // O_g at kOCol + g * D
+  static_assert(kOCol + kTcQTiles * D <= kTmemCols, "tensor-memory plan");
   static_assert(kSmemBytes <= 227 * 1024, "shared-memory plan");
 };
 
@@ -104,9 +116,9 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                            const __grid_constant__ CUtensorMap tmap_k,
-                            const __grid_constant__ CUtensorMap tmap_v,
-                            const PrefillParams p) {
+                         const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v,
+                         const PrefillParams p) {
   using TP = TcPlan<D>;
   constexpr int H = TP::kHalves;
 
@@ -114,16 +126,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base = (raw_u32 + 1023u) & ~1023u;
   uint8_t *base_ptr = smem_raw + (base - raw_u32);
-  const uint32_t sq = base;                        // Q half x at sq + x * kQHalfBytes
-  const uint32_t sring = base + TP::kStageOff;     // stage st at sring + st * kStageBytes
-  const uint32_t sp = base + TP::kPOff;            // P buffer b: high at sp + 2b kPBytes
+  const uint32_t sq = base;                        // Q of tile g, half x: sq + g kQBytes + x kQHalfBytes
+  const uint32_t sk = base + TP::kKOff;            // K stage st at sk + st * kTileBytes
+  const uint32_t sv = base + TP::kVOff;            // V stage st at sv + st * kTileBytes
   const uint32_t bar_q = base + TP::kBarOff;
-  const uint32_t bar_kv_full = bar_q + 8;
-  const uint32_t bar_kv_empty = bar_kv_full + 8 * kTcStages;
-  const uint32_t bar_s_full = bar_kv_empty + 8 * kTcStages;
-  const uint32_t bar_p_full = bar_s_full + 16;
-  const uint32_t bar_pv_done = bar_p_full + 16;
-  const uint32_t bar_drain = bar_pv_done + 16;
+  const uint32_t bar_k_full = bar_q + 8;
+  const uint32_t bar_k_empty = bar_k_full + 8 * kTcKStages;
+  const uint32_t bar_v_full = bar_k_empty + 8 * kTcKStages;
+  const uint32_t bar_v_empty = bar_v_full + 8 * kTcVStages;
+  const uint32_t bar_s_full = bar_v_empty + 8 * kTcVStages;   // [tile][2]
+  const uint32_t bar_p_full = bar_s_full + 16 * kTcQTiles;    // [tile][2]
+  const uint32_t bar_pv_done = bar_p_full + 16 * kTcQTiles;   // [tile][2]
+  const uint32_t bar_drain = bar_pv_done + 16 * kTcQTiles;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base_ptr + TP::kBarOff + 8 * TP::kNumBars);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -138,23 +152,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int q0 = p.query_start[s];
   const int n = min(p.query_start[s + 1] - q0, L);  // chunk length
   const int tpt = p.tokens_per_tile;
-  const int t0 = qt * tpt;                          // first chunk token of this tile
+  const int t0 = qt * kTcQTiles * tpt;              // first chunk token of this CTA
   if (t0 >= n) return;
   if (bad_len && threadIdx.x == 0 && qt == 0) raise_error(kErrContextClamp);
   const int group = p.group;
-  const int t1 = min(n, t0 + tpt);
   const int ctx0 = L - n;                           // position of chunk token 0
-  const int kmax = ctx0 + t1 - 1;                   // last key any row here sees
+  const bool has1 = t0 + tpt < n;                   // query tile 1 has tokens
+  // key tiles each query tile needs (keys up to its last token's position)
+  int nt_g[kTcQTiles];
+#pragma unroll
+  for (int g = 0; g < kTcQTiles; ++g) {
+    const int tb = t0 + g * tpt;
+    nt_g[g] = tb < n ? (ctx0 + min(n, tb + tpt) - 1) / kTcKeys + 1 : 0;
+  }
+  const int ntiles = has1 ? nt_g[1] : nt_g[0];      // key tiles the CTA streams
+  const int kmax = ctx0 + min(n, t0 + kTcQTiles * tpt) - 1;
   const int nblk = kmax / kBS + 1;
-  const int ntiles = kmax / kTcKeys + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(bar_kv_full + 8u * i, 1);
-      mbar_init(bar_kv_empty + 8u * i, 1);
+    for (int i = 0; i < kTcKStages; ++i) {
+      mbar_init(bar_k_full + 8u * i, 1);
+      mbar_init(bar_k_empty + 8u * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kTcVStages; ++i) {
+      mbar_init(bar_v_full + 8u * i, 1);
+      mbar_init(bar_v_empty + 8u * i, 1);
+    }
+    for (int i = 0; i < 2 * kTcQTiles; ++i) {
       mbar_init(bar_s_full + 8u * i, 1);
       mbar_init(bar_p_full + 8u * i, 4 * 32);
       mbar_init(bar_pv_done + 8u * i, 1);
@@ -172,16 +197,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == kTcProducerWarp) {
-    // ------------------------------------------------------------ producer
+  if (warp == kTcKWarp || warp == kTcVWarp) {
+    // ---------------------------------------------------------- producers
+    // warp kTcKWarp: Q, then K tiles into a 4-stage ring freed after S;
+    // warp kTcVWarp: V tiles into a 3-stage ring freed after PV.
+    const bool is_k = warp == kTcKWarp;
+    const int nst = is_k ? kTcKStages : kTcVStages;
+    const uint32_t ring = is_k ? sk : sv;
+    const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
+    const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
+    const CUtensorMap *tmap = is_k ? &tmap_k : &tmap_v;
     if (lane == 0) {
-      prefetch_tmap(&tmap_q);
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
-      mbar_arrive_expect_tx(bar_q, H * 128 * group * tpt);
+      prefetch_tmap(tmap);
+      if (is_k) {
+        prefetch_tmap(&tmap_q);
+        mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * H * 128 * group * tpt);
+        for (int g = 0; g < (has1 ? 2 : 1); ++g)
 #pragma unroll
-      for (int x = 0; x < H; ++x)
-        tma_load_3d(sq + x * TP::kQHalfBytes, &tmap_q, bar_q, 64 * x, h * group, q0 + t0);
+          for (int x = 0; x < H; ++x)
+            tma_load_3d(sq + g * TP::kQBytes + x * TP::kQHalfBytes, &tmap_q, bar_q, 64 * x,
+                        h * group, q0 + t0 + g * tpt);
+      }
     }
     const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
     const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
@@ -198,12 +234,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int b = 0; b < kTcBlocks; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, (j & 7) * kTcBlocks + b);
       if (lane == 0) {
-        const int st = j % kTcStages;
-        if (j >= kTcStages) ok = tc_wait(bar_kv_empty + 8u * st, ((j / kTcStages) - 1) & 1, s_abort);
+        const int st = j % nst;
+        if (j >= nst) ok = tc_wait(bar_empty + 8u * st, ((j / nst) - 1) & 1, s_abort);
         if (ok) {
-          const uint32_t full = bar_kv_full + 8u * st;
-          const uint32_t kst = sring + st * TP::kStageBytes;
-          mbar_arrive_expect_tx(full, TP::kStageBytes);
+          const uint32_t full = bar_full + 8u * st;
+          const uint32_t dst = ring + st * TP::kTileBytes;
+          mbar_arrive_expect_tx(full, TP::kTileBytes);
 #pragma unroll
           for (int b = 0; b < kTcBlocks; ++b) {
             const bool real = j * kTcBlocks + b < nblk;
@@ -215,10 +251,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               y = (phys[b] * p.num_kv_heads + h) * kBS;
             }
 #pragma unroll
-            for (int x = 0; x < H; ++x) {
-              tma_load_2d(kst + x * TP::kKVHalfBytes + b * 2048, &tmap_k, full, 64 * x, y);
-              tma_load_2d(kst + (H + x) * TP::kKVHalfBytes + b * 2048, &tmap_v, full, 64 * x, y);
-            }
+            for (int x = 0; x < H; ++x)
+              tma_load_2d(dst + x * TP::kKVHalfBytes + b * 2048, tmap, full, 64 * x, y);
           }
           issued = j + 1;
         }
@@ -226,11 +260,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (lane == 0) {
-      if (bad_id) raise_error(kErrBlockRange);
+      if (bad_id && is_k) raise_error(kErrBlockRange);
       // no bulk copy may still be landing when the CTA exits
-      mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
-      for (int j = max(0, issued - kTcStages); j < issued; ++j)
-        mbar_wait_bounded(bar_kv_full + 8u * (j % kTcStages), (j / kTcStages) & 1, kWaitLimitNs);
+      if (is_k) mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
+      for (int j = max(0, issued - nst); j < issued; ++j)
+        mbar_wait_bounded(bar_full + 8u * (j % nst), (j / nst) & 1, kWaitLimitNs);
     }
   } else if (warp == kTcMmaWarp) {
     // ----------------------------------------------------------------- MMA
@@ -238,44 +272,61 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t id_s = tc_idesc_bf16(kTcRows, kTcKeys, false);
       constexpr uint32_t id_pv = tc_idesc_bf16(kTcRows, D, true);
       bool ok = tc_wait(bar_q, 0, s_abort);
-      // S_j = Q K_j^T into S buffer j % 2
+      // S_gj = Q_g K_j^T into tile g's S buffer j % 2, for every tile that
+      // still needs key tile j
       auto issue_s = [&](int j) {
-        const int st = j % kTcStages;
-        ok = tc_wait(bar_kv_full + 8u * st, (j / kTcStages) & 1, s_abort);
+        const int st = j % kTcKStages;
+        ok = tc_wait(bar_k_full + 8u * st, (j / kTcKStages) & 1, s_abort);
         if (!ok) return;
         tc_fence_after_sync();
-        const uint32_t kst = sring + st * TP::kStageBytes;
-        const uint32_t d = tmem + (j & 1) * kTcKeys;
+        const uint32_t kst = sk + st * TP::kTileBytes;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks & 3) * 32;  // 16 dims = 32 bytes of the atom row
-          const uint64_t a = tc_desc_sw128(sq + (ks >> 2) * TP::kQHalfBytes + off, 16, 1024);
-          const uint64_t b = tc_desc_sw128(kst + (ks >> 2) * TP::kKVHalfBytes + off, 16, 1024);
-          tc_mma_ss(d, a, b, id_s, ks > 0);
+        for (int g = 0; g < kTcQTiles; ++g) {
+          if (j >= nt_g[g]) continue;
+          const uint32_t d = tmem + (2 * g + (j & 1)) * kTcKeys;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks & 3) * 32;  // 16 dims = 32 bytes of the atom row
+            const uint64_t a = tc_desc_sw128(sq + g * TP::kQBytes + (ks >> 2) * TP::kQHalfBytes + off,
+                                             16, 1024);
+            const uint64_t b = tc_desc_sw128(kst + (ks >> 2) * TP::kKVHalfBytes + off, 16, 1024);
+            tc_mma_ss(d, a, b, id_s, ks > 0);
+          }
+          tc_commit(bar_s_full + 8u * (2 * g + (j & 1)));
         }
-        tc_commit(bar_s_full + 8u * (j & 1));
+        tc_commit(bar_k_empty + 8u * st);
       };
       if (ok) issue_s(0);
       if (ok && ntiles > 1) issue_s(1);
       for (int j = 0; j < ntiles && ok; ++j) {
-        ok = tc_wait(bar_p_full + 8u * (j & 1), (j >> 1) & 1, s_abort);
+        // every tile's P_j (and the zeroed V rows) before any PV_j
+#pragma unroll
+        for (int g = 0; g < kTcQTiles; ++g)
+          if (ok && j < nt_g[g]) ok = tc_wait(bar_p_full + 8u * (2 * g + (j & 1)), (j >> 1) & 1, s_abort);
+        if (!ok) break;
+        const int st = j % kTcVStages;
+        ok = tc_wait(bar_v_full + 8u * st, (j / kTcVStages) & 1, s_abort);
         if (!ok) break;
         tc_fence_after_sync();
-        const int st = j % kTcStages;
-        const uint32_t vst = sring + st * TP::kStageBytes + H * TP::kKVHalfBytes;
-        const uint32_t pb = sp + (j & 1) * 2 * TP::kPBytes;
+        const uint32_t vst = sv + st * TP::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTcBlocks; ++kk) {
-          // V: 16 keys (two 8-key atoms, 1024 B apart) x head_dim (64-dim
-          // atoms kKVHalfBytes apart), dims contiguous
-          const uint64_t b = tc_desc_sw128(vst + kk * 2048, TP::kKVHalfBytes, 1024);
-          const uint64_t a_hi = tc_desc_sw128(pb + kk * 32, 16, 1024);
-          const uint64_t a_lo = tc_desc_sw128(pb + TP::kPBytes + kk * 32, 16, 1024);
-          tc_mma_ss(tmem + TP::kOCol, a_hi, b, id_pv, j > 0 || kk > 0);
-          tc_mma_ss(tmem + TP::kOCol, a_lo, b, id_pv, true);
+        for (int g = 0; g < kTcQTiles; ++g) {
+          if (j >= nt_g[g]) continue;
+          // P_gj (high, low) lives in S_gj's tensor-memory columns: 16 keys
+          // per 8 columns, high in the first 32 columns, low in the last 32
+          const uint32_t pt = tmem + (2 * g + (j & 1)) * kTcKeys;
+          const uint32_t o = tmem + TP::kOCol + g * D;
+#pragma unroll
+          for (int kk = 0; kk < kTcBlocks; ++kk) {
+            // V: 16 keys (two 8-key atoms, 1024 B apart) x head_dim (64-dim
+            // atoms kKVHalfBytes apart), dims contiguous
+            const uint64_t b = tc_desc_sw128(vst + kk * 2048, TP::kKVHalfBytes, 1024);
+            tc_mma_ts(o, pt + kk * 8, b, id_pv, j > 0 || kk > 0);
+            tc_mma_ts(o, pt + kTcKeys / 2 + kk * 8, b, id_pv, true);
+          }
+          tc_commit(bar_pv_done + 8u * (2 * g + (j & 1)));
         }
-        tc_commit(bar_pv_done + 8u * (j & 1));
-        tc_commit(bar_kv_empty + 8u * st);
+        tc_commit(bar_v_empty + 8u * st);
         if (j + 2 < ntiles) issue_s(j + 2);
       }
       // every MMA issued here has completed before tensor memory is freed
@@ -285,25 +336,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
-    const int r = warp * 32 + lane;               // row = tensor-memory lane
-    const int t = r / group;
-    const int nh = r - t * group;
-    const bool valid = t < tpt && t0 + t < n;
-    const int klim = valid ? ctx0 + t0 + t : -1;  // keys <= klim are visible
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    // the tile holding the context's last, partly filled block: zero the V
-    // rows past the context end (NaN allowed there) before PV reads them
+    const int g = warp >> 2;                      // query tile of this warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;            // row = tensor-memory lane
+    const int tl = r / group;
+    const int nh = r - tl * group;
+    const int tok = t0 + g * tpt + tl;            // chunk token of this row
+    const bool valid = tl < tpt && tok < n;
+    const int klim = valid ? ctx0 + tok : -1;     // keys <= klim are visible
+    const int ntg = nt_g[g];
+    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t ocol = TP::kOCol + g * D;
+    // the key tile holding the context's last, partly filled block: the
+    // warpgroup of the CTA's last query tile zeroes the V rows past the
+    // context end (NaN allowed there) before any PV reads them
     const int tail = L % kBS;
     const int zero_tile = (tail != 0 && (L - 1) / kBS < nblk) ? (L - 1) / kTcKeys : -1;
+    const bool zeroer = quarter == 0 && g == (has1 ? 1 : 0);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8u * (j & 1), (j >> 1) & 1, s_abort));
+    for (int j = 0; j < ntg; ++j) {
+      const int sb = 2 * g + (j & 1);
+      ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8u * sb, (j >> 1) & 1, s_abort));
       if (!ok) break;
       tc_fence_after_sync();
       uint32_t sr[2][32];
-      tc_ld_32x32b_x32(trow + (j & 1) * kTcKeys, sr[0]);
-      tc_ld_32x32b_x32(trow + (j & 1) * kTcKeys + 32, sr[1]);
+      tc_ld_32x32b_x32(trow + sb * kTcKeys, sr[0]);
+      tc_ld_32x32b_x32(trow + sb * kTcKeys + 32, sr[1]);
       tc_wait_ld();
       float z[kTcKeys];
       const int kb = j * kTcKeys;
@@ -328,60 +387,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool raise = m_new != m_used;
       const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        // O must hold PV_{j-1} before its rows are rescaled
-        ok = __all_sync(0xffffffffu,
-                        tc_wait(bar_pv_done + 8u * ((j - 1) & 1), ((j - 1) >> 1) & 1, s_abort));
+        // O_g must hold PV_{j-1} before its rows are rescaled
+        ok = __all_sync(0xffffffffu, tc_wait(bar_pv_done + 8u * (2 * g + ((j - 1) & 1)),
+                                             ((j - 1) >> 1) & 1, s_abort));
         if (!ok) break;
         tc_fence_after_sync();
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          tc_ld_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+          tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tc_st_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+          tc_st_32x32b_x32(trow + ocol + cc * 32, o);
         }
         tc_wait_st();
       }
       l *= alpha;
       m_used = m_new;
-      // P buffer j % 2 is free once PV_{j-2} has completed
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu,
-                        tc_wait(bar_pv_done + 8u * (j & 1), ((j - 2) >> 1) & 1, s_abort));
-        if (!ok) break;
-      }
-      const uint32_t phi = sp + (j & 1) * 2 * TP::kPBytes + r * 128;
-      const uint32_t plo = phi + TP::kPBytes;
+      // P replaces S in its tensor-memory columns: high parts in the first
+      // 32 columns, low parts in the last 32, two bf16 per column
       const bool live = valid && m_used != -INFINITY;
       float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t hi[kTcKeys / 2], lo[kTcKeys / 2];
 #pragma unroll
-      for (int q = 0; q < kTcKeys / 8; ++q) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = q * 8 + 2 * e;
-          const float p0 = live ? ex2_approx(z[c] - m_used) : 0.f;
-          const float p1 = live ? ex2_approx(z[c + 1] - m_used) : 0.f;
-          rsum[e] += p0 + p1;
-          hi[e] = pack2<false>(p0, p1);
-          float u0, u1;
-          unpack2<false>(hi[e], u0, u1);
-          lo[e] = pack2<false>(p0 - u0, p1 - u1);
-        }
-        const uint32_t chunk = static_cast<uint32_t>((q ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(phi + chunk), "r"(hi[0]),
-                     "r"(hi[1]), "r"(hi[2]), "r"(hi[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(plo + chunk), "r"(lo[0]),
-                     "r"(lo[1]), "r"(lo[2]), "r"(lo[3])
-                     : "memory");
+      for (int e = 0; e < kTcKeys / 2; ++e) {
+        const int c = 2 * e;
+        const float p0 = live ? ex2_approx(z[c] - m_used) : 0.f;
+        const float p1 = live ? ex2_approx(z[c + 1] - m_used) : 0.f;
+        rsum[e & 3] += p0 + p1;
+        hi[e] = pack2<false>(p0, p1);
+        float u0, u1;
+        unpack2<false>(hi[e], u0, u1);
+        lo[e] = pack2<false>(p0 - u0, p1 - u1);
       }
-      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
-      l += rs;
-      if (j == zero_tile && warp == 0) {
-        const uint32_t vb = sring + (j % kTcStages) * TP::kStageBytes + H * TP::kKVHalfBytes +
+      tc_st_32x32b_x32(trow + sb * kTcKeys, hi);
+      tc_st_32x32b_x32(trow + sb * kTcKeys + kTcKeys / 2, lo);
+      l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+      if (j == zero_tile && zeroer &&
+          __all_sync(0xffffffffu, tc_wait(bar_v_full + 8u * (j % kTcVStages),
+                                          (j / kTcVStages) & 1, s_abort))) {
+        // V_j has landed (its loads could otherwise overwrite the zeros)
+        const uint32_t vb = sv + (j % kTcVStages) * TP::kTileBytes +
                             (((L - 1) / kBS) % kTcBlocks) * 2048;
         const int nrow = kBS - tail;
         for (int i = lane; i < nrow * 8 * H; i += 32) {
@@ -390,23 +437,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t a = vb + (rem >> 3) * TP::kKVHalfBytes + row * 128 + (rem & 7) * 16;
           asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      tc_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(bar_p_full + 8u * (j & 1));
+      mbar_arrive(bar_p_full + 8u * sb);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok)
-      ok = __all_sync(0xffffffffu, tc_wait(bar_pv_done + 8u * ((ntiles - 1) & 1),
-                                           ((ntiles - 1) >> 1) & 1, s_abort));
-    if (ok) {
+    if (ok && ntg > 0)
+      ok = __all_sync(0xffffffffu, tc_wait(bar_pv_done + 8u * (2 * g + ((ntg - 1) & 1)),
+                                           ((ntg - 1) >> 1) & 1, s_abort));
+    if (ok && ntg > 0) {
       tc_fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float *orow = p.out + (static_cast<int64_t>(q0 + t0 + t) * p.num_q_heads + h * group + nh) * D;
+      float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        tc_ld_32x32b_x32(trow + TP::kOCol + cc * 32, o);
+        tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
         tc_wait_ld();
         if (valid) {
 #pragma unroll
