@@ -137,3 +137,29 @@ def test_swap_rejects_bad_arguments_on_host(kw, expect):
              dnb=8, stream=None)
     a.update(kw)
     assert _lib.lib().pa_swap_blocks(*a.values()) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(T=0), OK),                        # nothing to launch
+    (dict(S=0), OK),
+    (dict(maxq=0), OK),
+    (dict(dtype=1), UNSUPPORTED),           # fp8 caches: decode only
+    (dict(dtype=7), INVALID),
+    (dict(B=8), UNSUPPORTED),
+    (dict(D=96), UNSUPPORTED),
+    (dict(Hq=12, Hkv=8), UNSUPPORTED),      # not a whole group
+    (dict(Hq=32, Hkv=1), UNSUPPORTED),      # group 32 > 16
+    (dict(scale=float("inf")), INVALID),
+    (dict(NB=0), INVALID),
+    (dict(maxb=-1), INVALID),
+    (dict(out=None), INVALID),
+    (dict(qs=None), INVALID),
+    (dict(out=FAKE + 4), INVALID),          # misaligned
+    (dict(k=FAKE + 8), INVALID),
+])
+def test_prefill_rejects_bad_arguments_on_host(kw, expect):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, dtype=0, bt=FAKE, maxb=8, qs=FAKE, cl=FAKE,
+             maxq=64, maxctx=128, S=2, T=100, Hq=8, Hkv=2, D=128, B=16, NB=64, scale=0.1,
+             stream=None)
+    a.update(kw)
+    assert _lib.lib().pa_prefill(*a.values()) == expect

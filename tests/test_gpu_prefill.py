@@ -18,6 +18,7 @@ from paged_kv_cache_429_b200.batch import DecodeBatch
 from parity_harness import BF16_TOL, oracle_caches, to_u16
 
 pytestmark = pytest.mark.gpu
+PA_DEVERR_BLOCK_RANGE = 0x10
 
 
 @pytest.fixture(autouse=True)
@@ -95,3 +96,44 @@ def test_prefill_leaves_rows_outside_the_chunks_alone():
     torch.cuda.synchronize()
     assert torch.all(big[:4] == 5.0) and torch.all(big[-4:] == 5.0)
     assert torch.all(torch.isfinite(out))
+
+
+def test_block_id_outside_pool_reads_zeros_and_is_flagged():
+    """Table entries outside [0, num_blocks) read as zero K/V and set
+    PA_DEVERR_BLOCK_RANGE; other sequences are unaffected."""
+    lens, chunks = [40, 200, 90], [40, 64, 30]
+    b, q, qs = build(8, 2, 128, lens, chunks, seed=4)
+    good = run_prefill(b, q, qs, chunks)
+    assert pa_get_device_error() == 0
+    bt = b.block_tables.clone()
+    bt[0, 1] = b.num_blocks + 3
+    bt[1, 0] = -7
+    out = torch.full_like(good, float("nan"))
+    pa_prefill(out, q, b.k_cache, b.v_cache, bt, torch.from_numpy(qs).cuda(), b.context_lens,
+               int(max(chunks)), b.max_context_len, b.w.sm_scale)
+    torch.cuda.synchronize()
+    assert pa_get_device_error() & PA_DEVERR_BLOCK_RANGE
+    assert torch.all(torch.isfinite(out))
+    s2 = slice(int(qs[2]), int(qs[3]))
+    assert torch.equal(out[s2], good[s2])
+    # the oracle with those blocks' K/V zeroed gives the same answer
+    kc, vc = oracle_caches(b)
+    tables = b.tables.copy()
+    zero_id = b.num_blocks  # an extra all-zero block appended to the caches
+    kc = np.concatenate([kc, np.zeros_like(kc[:1])])
+    vc = np.concatenate([vc, np.zeros_like(vc[:1])])
+    tables[0, 1] = zero_id
+    tables[1, 0] = zero_id
+    ref = oracle.paged_prefill(to_u16(q), kc, vc, tables, qs, b.lens.astype(np.int32),
+                               b.w.sm_scale)
+    assert float(np.max(np.abs(out.double().cpu().numpy() - ref))) <= BF16_TOL
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_mha_long_chunks_span_many_query_tiles(d):
+    """Group 1 (128 tokens per query tile, 256 per CTA): chunks that end
+    inside the first or the second tile of a CTA and span several CTAs."""
+    lens = [1500, 700, 257, 129]
+    chunks = [1500, 300, 257, 128]
+    b, q, qs = build(4, 4, d, lens, chunks, seed=5)
+    check(b, q, qs, chunks)
