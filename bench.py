@@ -69,11 +69,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank space, so that the hash
+    changes with the compiled code only."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
 def decode_source_hash() -> str:
     h = hashlib.sha256()
     for rel in DECODE_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

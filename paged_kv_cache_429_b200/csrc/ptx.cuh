@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA
-// tiled loads (no multicast), ldmatrix / movmatrix, warp-level bf16/f16 MMA,
+// tiled loads (each CTA loads its own tiles), ldmatrix / movmatrix, warp-level bf16/f16 MMA,
 // the fp8 E4M3 -> f16 conversion, and the 5th-generation tensor core
 // (tcgen05: tensor-memory allocation, MMA, commit, loads and stores).
 #pragma once
@@ -90,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // ---------------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar`.
-// Plain per-CTA load: no cluster multicast.
+// Plain per-CTA load into this CTA's own shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap,
                                             uint32_t bar, int x, int y) {
   asm volatile(
