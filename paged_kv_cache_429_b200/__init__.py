@@ -29,7 +29,7 @@ from ._lib import STATUS_NAMES, LibraryNotBuilt
 
 __all__ = [
     "PA_KV_BF16", "PA_KV_FP8_E4M3", "BLOCK_SIZE", "PagedAttentionError",
-    "LibraryNotBuilt", "pa_decode", "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks",
+    "LibraryNotBuilt", "pa_decode", "pa_decode_no_alloc", "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks",
     "pa_swap_blocks", "pa_decode_workspace_size", "pa_get_device_error",
     "pa_status_string",
     "BlockPool", "kv_dtype_of",
@@ -126,6 +126,37 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
         int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode")
+    return out
+
+
+def pa_decode_no_alloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                       v_cache: torch.Tensor, block_tables: torch.Tensor,
+                       context_lens: torch.Tensor, max_context_len: int, sm_scale: float,
+                       *, k_scale: float = 1.0, v_scale: float = 1.0,
+                       partition_size: int = 512,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Split-context decode with the library's own fixed scratch (see pa.h:
+    no allocation; launches needing more than PA_NO_ALLOC_SCRATCH_BYTES are
+    refused; calls overlapping on the GPU race on the scratch)."""
+    _need(out, "out", (torch.float32,), 3)
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.float8_e4m3fn, torch.uint8), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_tables, "block_tables", (torch.int32,), 2)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    S, Hq, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    if tuple(out.shape) != (S, Hq, D) or Dc != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between out, q and the caches")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables / context_lens must have num_seqs rows")
+    rc = _lib.lib().pa_decode_no_alloc(
+        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+        kv_dtype_of(k_cache), float(k_scale), float(v_scale),
+        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+        int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
+        int(partition_size), _stream_ptr(stream, q.device))
+    _ok(rc, "pa_decode_no_alloc")
     return out
 
 
