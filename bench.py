@@ -235,6 +235,7 @@ def run_ours(args, world, rank, local):
     eb = 1 if w.kv_fp8 else 2
     reshape_bytes = step_writes * w.num_kv_heads * w.head_dim * (2 * 2 + 2 * eb) + 8 * step_writes
     decode_bytes = batch.algorithmic_bytes()
+    unique_kv = batch.unique_kv_bytes() if w.prefix_len else 0
     step_bytes = decode_bytes + reshape_bytes
     n_copy_launches = sum(1 for op in batch.step_ops if op.kind == "copy")
     n_write_launches = sum(1 for op in batch.step_ops if op.kind == "write")
@@ -308,6 +309,9 @@ def run_ours(args, world, rank, local):
             "seed": args.seed,
         },
         "tokens_per_s": round(w.num_seqs * world / (ms_per_step * 1e-3), 1),
+        **({"unique_kv_bytes_per_step": unique_kv,
+            "unique_kv_gbs": round(unique_kv * world / (ms_per_step * 1e-3) / 1e9, 2)}
+           if w.prefix_len else {}),
         "pct_of_peak": round(100 * value / world / peak, 2),
         "pct_of_8tbs_datasheet": round(100 * value / world / 8000.0, 2),
         "e2e": e2e,

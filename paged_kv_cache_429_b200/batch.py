@@ -209,3 +209,17 @@ class DecodeBatch:
         qo = w.num_seqs * w.num_q_heads * w.head_dim * (2 + 4)
         bt = int((-(-self.lens // BS)).sum()) * 4 + 4 * w.num_seqs
         return kv + qo + bt
+
+    def unique_kv_bytes(self) -> int:
+        """K and V bytes of the distinct physical blocks the step reads (a
+        block shared by several sequences counted once, with the most
+        tokens any of them uses in it)."""
+        w = self.w
+        eb = 1 if w.kv_fp8 else 2
+        used = {}
+        for s in range(w.num_seqs):
+            L = int(self.lens[s])
+            for j in range(-(-L // BS)):
+                p = int(self.tables[s][j])
+                used[p] = max(used.get(p, 0), min(BS, L - BS * j))
+        return sum(used.values()) * w.num_kv_heads * w.head_dim * eb * 2

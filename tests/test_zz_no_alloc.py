@@ -71,3 +71,16 @@ def test_scratch_larger_than_the_array_is_refused():
     # a bad partition size is an argument error
     assert call_no_alloc(b, out, 0) == 1 and call_no_alloc(b, out, 100) == 1
     assert np.all(out.cpu().numpy() == 7.0)
+
+
+def test_python_binding_matches_the_c_call():
+    from paged_kv_cache_429_b200 import pa_decode_no_alloc
+    b = DecodeBatch.build(synth.WORKLOADS["tiny"], 3)
+    b.step(partition_size=0)
+    a = torch.full_like(b.out, float("nan"))
+    assert call_no_alloc(b, a, 64) == 0
+    c = torch.full_like(b.out, float("nan"))
+    pa_decode_no_alloc(c, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+                       b.max_context_len, b.w.sm_scale, partition_size=64)
+    torch.cuda.synchronize()
+    assert torch.equal(a, c)
