@@ -44,6 +44,7 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20
 DECODE_SOURCES = ["paged_kv_cache_429_b200/csrc/decode.cuh",
+                  "paged_kv_cache_429_b200/csrc/kv_quant.cuh",
                   "paged_kv_cache_429_b200/csrc/ptx.cuh"]
 
 
@@ -240,17 +241,27 @@ def run_ours(args, world, rank, local):
     n_copy_launches = sum(1 for op in batch.step_ops if op.kind == "copy")
     n_write_launches = sum(1 for op in batch.step_ops if op.kind == "write")
 
+    fuse = not args.no_fuse
+
     def one_step(ev=None):
-        batch.run_ops(batch.step_ops)
-        if ev is not None:
-            ev[0].record(stream)
-        batch.decode(partition_size=ps, workspace=ws)
+        if fuse:
+            # copy-on-write copies, then one decode launch that also writes
+            # the new tokens (events bracket both: the decode launch and any
+            # copies in front of it)
+            if ev is not None:
+                ev[0].record(stream)
+            batch.step_fused(partition_size=ps, workspace=ws)
+        else:
+            batch.run_ops(batch.step_ops)
+            if ev is not None:
+                ev[0].record(stream)
+            batch.decode(partition_size=ps, workspace=ws)
         if ev is not None:
             ev[1].record(stream)
 
     # which decode path runs (split launches a second, reduce kernel)
     split = ps > 0 or (ps < 0 and ws is not None and _auto_split(batch, ws))
-    launches_per_step = n_write_launches + n_copy_launches + (2 if split else 1)
+    launches_per_step = (0 if fuse else n_write_launches) + n_copy_launches + (2 if split else 1)
 
     for _ in range(args.warmup):
         one_step()
@@ -292,7 +303,9 @@ def run_ours(args, world, rank, local):
     if rank != 0:
         return None
     peak, peak_src = measured_peak()
-    achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+    # the fused launch also reads and writes the step's new tokens
+    kernel_bytes = decode_bytes + (reshape_bytes if fuse else 0)
+    achieved = kernel_bytes / (dec_avg_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
@@ -303,6 +316,8 @@ def run_ours(args, world, rank, local):
             "seq_len": f"U[{w.len_lo},{w.len_hi}]" if not w.prefix_len else "prefix+suffix",
             "parallelism": f"dp{world} (independent sequence shards, no collective)",
             "decode_path": "split-context" if split else "single-pass",
+            "new_token_write": "fused into the decode launch (pa_decode_append)" if fuse
+                               else "separate pa_reshape_and_cache launch",
             "partition_size": ps,
             "l2": (f"inputs larger than L2: {decode_bytes / 1e9:.2f} GB per step vs "
                    f"{L2_BYTES / 2**20:.0f} MiB L2; no flush"),
@@ -319,8 +334,9 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(w.name),
-                     "kernel": "paged_decode_kernel" + (" + reduce" if split else ""),
-                     "algorithmic_bytes_per_launch": decode_bytes,
+                     "kernel": "paged_decode_kernel" + (" (new-token write fused)" if fuse else "")
+                               + (" + reduce" if split else ""),
+                     "algorithmic_bytes_per_launch": kernel_bytes,
                      "avg_launch_ms": round(dec_avg_ms, 6), "peak_source": peak_src},
         "clocks": clocks.summary(),
     }
@@ -345,8 +361,10 @@ def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):
     lengths; packed in one pinned buffer) host -> device and its output
     device -> host. Two slots of device buffers let step i+1's upload and
     step i-1's download run on their own streams while step i computes."""
-    from paged_kv_cache_429_b200 import pa_copy_blocks, pa_decode, pa_reshape_and_cache
+    from paged_kv_cache_429_b200 import (pa_copy_blocks, pa_decode, pa_decode_append,
+                                         pa_reshape_and_cache)
     b = batch
+    fuse = not args.no_fuse
     items = [("q", b.q), ("k_new", b.k_new), ("v_new", b.v_new),
              ("tables", b.block_tables), ("lens", b.context_lens)]
     for i, op in enumerate(b.step_ops):
@@ -390,15 +408,21 @@ def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):
         stream.wait_event(sl["up"])
         stream.wait_event(sl["down"])           # the slot's last output has been read back
         for j, op in enumerate(b.step_ops):
-            if op.kind == "write":
+            if op.kind == "copy":
+                pa_copy_blocks(b.k_cache, b.v_cache, v[f"pairs{j}"], stream=stream)
+            elif not fuse:
                 pa_reshape_and_cache(v["k_new"][op.row0:op.row1], v["v_new"][op.row0:op.row1],
                                      b.k_cache, b.v_cache, v[f"slots{j}"], k_scale=b.k_scale,
                                      v_scale=b.v_scale, stream=stream)
-            else:
-                pa_copy_blocks(b.k_cache, b.v_cache, v[f"pairs{j}"], stream=stream)
-        pa_decode(sl["out"], v["q"], b.k_cache, b.v_cache, v["tables"], v["lens"],
-                  b.max_context_len, b.w.sm_scale, k_scale=b.k_scale, v_scale=b.v_scale,
-                  partition_size=ps, workspace=ws, stream=stream)
+        if fuse:
+            pa_decode_append(sl["out"], v["q"], v["k_new"], v["v_new"], b.k_cache, b.v_cache,
+                             v["tables"], v["lens"], b.max_context_len, b.w.sm_scale,
+                             k_scale=b.k_scale, v_scale=b.v_scale, partition_size=ps,
+                             workspace=ws, stream=stream)
+        else:
+            pa_decode(sl["out"], v["q"], b.k_cache, b.v_cache, v["tables"], v["lens"],
+                      b.max_context_len, b.w.sm_scale, k_scale=b.k_scale, v_scale=b.v_scale,
+                      partition_size=ps, workspace=ws, stream=stream)
         sl["done"].record(stream)
         down_stream.wait_event(sl["done"])
         with torch.cuda.stream(down_stream):
@@ -656,6 +680,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fuse", action="store_true",
+                    help="write the new tokens with a separate pa_reshape_and_cache launch")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

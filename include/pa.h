@@ -134,6 +134,33 @@ PA_API pa_status pa_decode(float *out, const void *q, const void *k_cache,
                     int num_blocks, float sm_scale, int partition_size,
                     void *workspace, size_t workspace_bytes, void *stream);
 
+/* One decode step with the new tokens' cache write fused in: for every
+ * sequence s with L = context_lens[s] >= 1, writes key[s] / value[s] (the
+ * step's new token, at position L - 1) into slot
+ * block_tables[s][(L - 1) / 16] * 16 + (L - 1) % 16 of the caches exactly
+ * as pa_reshape_and_cache would (bf16 bits, or E4M3(x / scale) with the
+ * given k_scale / v_scale), then computes the same output as pa_decode —
+ * in the decode launch itself, which writes the token before it reads that
+ * block ([Ch7] §7.1 "Block 与 Block Table": a generated token goes into the
+ * next slot of the sequence's last block). The pages have no separate call
+ * for this; it saves the cache-write launch of every decode step. Any
+ * copy-on-write copy of a shared last block (pa_copy_blocks) must come
+ * first.
+ *   key, value   bf16 [num_seqs][num_kv_heads][head_dim], 16-byte aligned.
+ *   k_cache, v_cache  written in place (the new slots only).
+ *   Other arguments as for pa_decode. A table entry outside the pool is
+ *   not written (and reads as zeros, flagged PA_DEVERR_BLOCK_RANGE); a
+ *   clamped context length (PA_DEVERR_CONTEXT_CLAMP) writes nothing. */
+PA_API pa_status pa_decode_append(float *out, const void *q, const void *key,
+                                  const void *value, void *k_cache, void *v_cache,
+                                  pa_kv_dtype kv_dtype, float k_scale, float v_scale,
+                                  const int32_t *block_tables, int max_blocks_per_seq,
+                                  const int32_t *context_lens, int max_context_len,
+                                  int num_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int block_size, int num_blocks,
+                                  float sm_scale, int partition_size, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
 /* Split-context decode for callers that cannot allocate device memory.
  * The pages have no counterpart of this call; it exists for the runtime
  * around the kernels. Some callers have no device allocator to hand: a C

@@ -5,6 +5,7 @@ of libpa.so; PyTorch is used for device memory, streams and dtypes. The
 functions carry the names of the C entry points (include/pa.h):
 
     pa_decode               decode-step attention through block tables
+    pa_decode_append        the same with the step's new tokens written to their slots in-kernel
     pa_prefill              chunked causal prefill attention through block tables
     pa_reshape_and_cache    scatter new K/V into cache slots (bf16 / fp8)
     pa_copy_blocks          copy-on-write block copies
@@ -29,7 +30,7 @@ from ._lib import STATUS_NAMES, LibraryNotBuilt
 
 __all__ = [
     "PA_KV_BF16", "PA_KV_FP8_E4M3", "BLOCK_SIZE", "PagedAttentionError",
-    "LibraryNotBuilt", "pa_decode", "pa_decode_no_alloc", "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks",
+    "LibraryNotBuilt", "pa_decode", "pa_decode_append", "pa_decode_no_alloc", "pa_prefill", "pa_reshape_and_cache", "pa_copy_blocks",
     "pa_swap_blocks", "pa_decode_workspace_size", "pa_get_device_error",
     "pa_status_string",
     "BlockPool", "kv_dtype_of",
@@ -126,6 +127,48 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
         int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode")
+    return out
+
+
+def pa_decode_append(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor,
+                     value: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     block_tables: torch.Tensor, context_lens: torch.Tensor,
+                     max_context_len: int, sm_scale: float, *, k_scale: float = 1.0,
+                     v_scale: float = 1.0, partition_size: int = -1,
+                     workspace: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode step with the new tokens' cache write fused in (see pa.h):
+    key / value bf16 [S][Hkv][D] go to slot L - 1 of each sequence, then the
+    decode runs; out[S][Hq][D] fp32 is written in place."""
+    _need(out, "out", (torch.float32,), 3)
+    _need(q, "q", (torch.bfloat16,), 3)
+    _need(key, "key", (torch.bfloat16,), 3)
+    _need(value, "value", (torch.bfloat16,), 3)
+    _need(k_cache, "k_cache", (torch.bfloat16, torch.float8_e4m3fn, torch.uint8), 4)
+    _need(v_cache, "v_cache", (k_cache.dtype,), 4)
+    _need(block_tables, "block_tables", (torch.int32,), 2)
+    _need(context_lens, "context_lens", (torch.int32,), 1)
+    S, Hq, D = q.shape
+    NB, Hkv, B, Dc = k_cache.shape
+    if tuple(out.shape) != (S, Hq, D) or Dc != D or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("shape mismatch between out, q and the caches")
+    if tuple(key.shape) != (S, Hkv, D) or tuple(value.shape) != (S, Hkv, D):
+        raise ValueError("key / value must be [num_seqs][num_kv_heads][head_dim]")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables / context_lens must have num_seqs rows")
+    if workspace is None and partition_size != 0:
+        nbytes = pa_decode_workspace_size(S, Hq, D, max_context_len, partition_size)
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = _lib.lib().pa_decode_append(
+        out.data_ptr(), q.data_ptr(), key.data_ptr(), value.data_ptr(), k_cache.data_ptr(),
+        v_cache.data_ptr(), kv_dtype_of(k_cache), float(k_scale), float(v_scale),
+        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+        int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale), int(partition_size),
+        ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
+    _ok(rc, "pa_decode_append")
     return out
 
 

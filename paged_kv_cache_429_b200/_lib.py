@@ -26,6 +26,9 @@ SIGNATURES = {
     "pa_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _i32, _vp,
                          _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32,
                          _vp, _sz, _vp]),
+    "pa_decode_append": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _i32,
+                                _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                _f32, _i32, _vp, _sz, _vp]),
     "pa_decode_no_alloc": (_i32, [_vp, _vp, _vp, _vp, _i32, _f32, _f32, _vp, _i32,
                                   _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                   _f32, _i32, _vp]),

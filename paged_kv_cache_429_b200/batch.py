@@ -23,7 +23,7 @@ import torch
 
 import synth
 
-from . import (BlockPool, pa_copy_blocks, pa_decode, pa_decode_workspace_size,
+from . import (BlockPool, pa_copy_blocks, pa_decode, pa_decode_append, pa_decode_workspace_size,
                pa_reshape_and_cache)
 
 BS = 16
@@ -198,6 +198,24 @@ class DecodeBatch:
         """One decode step: write the new tokens (after any CoW copy), decode."""
         self.run_ops(self.step_ops, stream=stream)
         return self.decode(partition_size=partition_size, workspace=workspace, stream=stream)
+
+    def step_fused(self, partition_size: Optional[int] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """The same step with the new tokens' write fused into the decode
+        launch (pa_decode_append): any copy-on-write copies first, then one
+        decode that writes each sequence's new token before reading it."""
+        writes = [op for op in self.step_ops if op.kind == "write"]
+        assert len(writes) == 1 and writes[0].src == "new" and writes[0].row0 == 0 \
+            and writes[0].row1 == self.w.num_seqs
+        for op in self.step_ops:
+            if op.kind == "copy":
+                pa_copy_blocks(self.k_cache, self.v_cache, self._dev_pairs[id(op)], stream=stream)
+        ps = self.w.partition_size if partition_size is None else partition_size
+        return pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.k_cache,
+                                self.v_cache, self.block_tables, self.context_lens,
+                                self.max_context_len, self.w.sm_scale, k_scale=self.k_scale,
+                                v_scale=self.v_scale, partition_size=ps, workspace=workspace,
+                                stream=stream)
 
     # ---------------------------------------------------------- accounting
     def algorithmic_bytes(self) -> int:

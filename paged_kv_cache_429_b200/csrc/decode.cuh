@@ -37,6 +37,9 @@
 //     either the normalised output (single-pass) or the partition's
 //     unnormalised output with its max and sum (split; a second kernel
 //     combines the partitions).
+// With the step's new tokens fused in (pa_decode_append), the CTA holding a
+// sequence's last block first writes the new token's K/V row of its KV head
+// into slot L - 1 (as reshape_and_cache would), then streams as above.
 // fp8 E4M3 caches are widened to f16 exactly (cvt.rn.f16x2.e4m3x2) and use
 // the f16 MMA; q is then scaled per head by a power of two into f16 range
 // (exact), and the power is divided out of the scores.
@@ -45,6 +48,7 @@
 #include <cuda.h>
 #include <cstdint>
 
+#include "kv_quant.cuh"
 #include "ptx.cuh"
 
 namespace pa {
@@ -131,6 +135,16 @@ struct DecodeParams {
   int max_partitions;           // P (workspace stride)
   float score_scale;            // sm_scale * log2(e) [* k_scale for fp8]
   float out_scale;              // v_scale for fp8, 1 for bf16
+  // fused write of the step's new token (append != 0): sequence s's new K
+  // and V rows (bf16 [S][Hkv][D]) go to slot L_s - 1 of its table before
+  // anything reads that block
+  int append;
+  const uint16_t *new_k;
+  const uint16_t *new_v;
+  void *k_cache;
+  void *v_cache;
+  float k_scale;                // fp8 quantisation scales of the new rows
+  float v_scale;
 };
 
 __device__ unsigned int g_pa_error;
@@ -549,6 +563,33 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
     const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
+    // Fused write of the step's new token (pa_decode_append): the CTA whose
+    // range holds the token's block writes the token's K and V rows of this
+    // KV head (one 8-element chunk per lane). The rows are loaded at once,
+    // stored once the first stage's loads are issued (so their latency does
+    // not hold up the stream), and fenced against the TMA reads right before
+    // the load of the token's block. An id outside the pool is left alone
+    // (its loads read zeros and are flagged below).
+    int write_stage = -1;  // ring stage holding the new token's block
+    bool pending = false;  // this lane has a chunk to store
+    uint4 new_kx = make_uint4(0u, 0u, 0u, 0u), new_vx = new_kx;
+    int64_t new_dst = 0;
+    if (p.append && L > 0 && !bad_len) {
+      const int jl = (L - 1) / kBS;
+      if (jl >= j0 && jl < j1) {
+        write_stage = (jl - j0) / BPS;
+        const int pid = bt[jl];
+        if (lane < D / 8 && pid >= 0 && pid < p.num_blocks) {
+          const int64_t src = (static_cast<int64_t>(s) * p.num_kv_heads + h) * D + lane * 8;
+          new_kx = *reinterpret_cast<const uint4 *>(p.new_k + src);
+          new_vx = *reinterpret_cast<const uint4 *>(p.new_v + src);
+          new_dst = ((static_cast<int64_t>(pid) * p.num_kv_heads + h) * kBS + (L - 1) % kBS) * D +
+                    lane * 8;
+          pending = true;
+        }
+      }
+    }
+    bool stored = false;
     int issued = 0;
     bool ok = true;
     bool bad_id = false;
@@ -561,6 +602,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
         int phys[BPS];
 #pragma unroll
         for (int b = 0; b < BPS; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, i * BPS + b - jb);
+        if (pending && !stored && (i > 0 || i == write_stage)) {
+          store_kv_chunk<FP8>(new_kx, new_vx, p.k_cache, p.v_cache, new_dst, p.k_scale,
+                              p.v_scale);
+          stored = true;
+        }
+        if (i == write_stage) {  // the new token's row is stored before its block is read
+          if (stored) fence_proxy_async_global();
+          __syncwarp();
+        }
         if (lane == 0) {
           const int st = i % NS;
           if (i >= NS && !mbar_try_wait(empty0 + 8u * st, ((i / NS) - 1) & 1)) {

@@ -192,13 +192,17 @@ size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim,
   return workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_context_len, psize);
 }
 
-pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
-                    pa_kv_dtype kv_dtype, float k_scale, float v_scale,
-                    const int32_t *block_tables, int max_blocks_per_seq,
-                    const int32_t *context_lens, int max_context_len, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int num_blocks, float sm_scale, int partition_size, void *workspace,
-                    size_t workspace_bytes, void *stream) {
+// pa_decode, and with new_k / new_v set pa_decode_append (the step's new
+// tokens written by the decode kernel itself).
+static pa_status decode_common(float *out, const void *q, const void *k_cache,
+                               const void *v_cache, pa_kv_dtype kv_dtype, float k_scale,
+                               float v_scale, const int32_t *block_tables,
+                               int max_blocks_per_seq, const int32_t *context_lens,
+                               int max_context_len, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               float sm_scale, int partition_size, void *workspace,
+                               size_t workspace_bytes, void *stream, const void *new_k,
+                               const void *new_v) {
   // ---- shape and pointer checks (host only; nothing launched on error)
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       max_blocks_per_seq < 0 || max_context_len < 0 || num_blocks <= 0)
@@ -219,6 +223,8 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return PA_ERR_INVALID_ARG;
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return PA_ERR_INVALID_ARG;
+  if ((new_k || new_v) && !(new_k && new_v && aligned(new_k, 16) && aligned(new_v, 16)))
     return PA_ERR_INVALID_ARG;
   const int64_t rows64 = static_cast<int64_t>(num_blocks) * num_kv_heads * pa::kBS;
   if (rows64 + pa::kBS >= INT32_MAX) return PA_ERR_UNSUPPORTED;
@@ -267,6 +273,15 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   p.num_kv_heads = num_kv_heads;
   p.group = group;
   p.num_blocks = num_blocks;
+  if (new_k) {
+    p.append = 1;
+    p.new_k = static_cast<const uint16_t *>(new_k);
+    p.new_v = static_cast<const uint16_t *>(new_v);
+    p.k_cache = const_cast<void *>(k_cache);
+    p.v_cache = const_cast<void *>(v_cache);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+  }
   const float log2e = 1.4426950408889634f;
   if (kv_dtype == PA_KV_BF16) {
     p.score_scale = sm_scale * log2e;
@@ -327,6 +342,34 @@ pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *
   r.max_partitions = static_cast<int>(P);
   return head_dim == 128 ? launch_reduce<128>(r, num_seqs, st)
                          : launch_reduce<64>(r, num_seqs, st);
+}
+
+pa_status pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+                    pa_kv_dtype kv_dtype, float k_scale, float v_scale,
+                    const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, int max_context_len, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float sm_scale, int partition_size, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  return decode_common(out, q, k_cache, v_cache, kv_dtype, k_scale, v_scale, block_tables,
+                       max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, sm_scale, partition_size,
+                       workspace, workspace_bytes, stream, nullptr, nullptr);
+}
+
+pa_status pa_decode_append(float *out, const void *q, const void *key, const void *value,
+                           void *k_cache, void *v_cache, pa_kv_dtype kv_dtype, float k_scale,
+                           float v_scale, const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int max_context_len, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float sm_scale, int partition_size, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+  if (num_seqs > 0 && (!key || !value)) return PA_ERR_INVALID_ARG;
+  return decode_common(out, q, k_cache, v_cache, kv_dtype, k_scale, v_scale, block_tables,
+                       max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, sm_scale, partition_size,
+                       workspace, workspace_bytes, stream, num_seqs > 0 ? key : nullptr,
+                       num_seqs > 0 ? value : nullptr);
 }
 
 pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cache,

@@ -163,3 +163,20 @@ def test_prefill_rejects_bad_arguments_on_host(kw, expect):
              stream=None)
     a.update(kw)
     assert _lib.lib().pa_prefill(*a.values()) == expect
+
+
+def declared_arity():
+    """Parameter count of every PA_API function in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"PA_API[^;(]*?\b(pa_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [p for p in m.group(2).split(",") if p.strip()]
+        out[m.group(1)] = 0 if params == ["void"] or [p.strip() for p in params] == ["void"] \
+            else len(params)
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    arity = declared_arity()
+    for name, (_, args) in _lib.SIGNATURES.items():
+        assert len(args) == arity[name], (name, len(args), arity[name])
