@@ -241,7 +241,7 @@ def run_ours(args, world, rank, local):
     n_copy_launches = sum(1 for op in batch.step_ops if op.kind == "copy")
     n_write_launches = sum(1 for op in batch.step_ops if op.kind == "write")
 
-    fuse = not args.no_fuse
+    fuse = args.fuse
 
     def one_step(ev=None):
         if fuse:
@@ -364,7 +364,7 @@ def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):
     from paged_kv_cache_429_b200 import (pa_copy_blocks, pa_decode, pa_decode_append,
                                          pa_reshape_and_cache)
     b = batch
-    fuse = not args.no_fuse
+    fuse = args.fuse
     items = [("q", b.q), ("k_new", b.k_new), ("v_new", b.v_new),
              ("tables", b.block_tables), ("lens", b.context_lens)]
     for i, op in enumerate(b.step_ops):
@@ -680,8 +680,9 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-fuse", action="store_true",
-                    help="write the new tokens with a separate pa_reshape_and_cache launch")
+    ap.add_argument("--fuse", action="store_true",
+                    help="write the new tokens inside the decode launch (pa_decode_append) "
+                         "instead of a separate pa_reshape_and_cache launch")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

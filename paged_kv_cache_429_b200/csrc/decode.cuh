@@ -97,7 +97,12 @@ struct Plan {
   static constexpr int kMergeBytes = 2 * 32 * kLaneFloats * 4;  // warps 2 and 3
   static constexpr int kMergeOffset = CHUNKED ? kRingBytes : 0;
   static constexpr int kBarOffset = CHUNKED ? kRingBytes + kMergeBytes : kRingBytes;
-  static constexpr int kSmemBytes = 1024 + kBarOffset + 16 * kStages + 16;
+  // the step's new K and V rows (bf16) for the fused cache write, then a
+  // word saying whether their block id is inside the pool
+  static constexpr int kPatchOffset = kBarOffset + 16 * kStages + 16;
+  static constexpr int kSmemBytes = 1024 + kPatchOffset + 4 * D + 16;
+  // 3 CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+  static_assert(NT == 2 || 3 * (kSmemBytes + 1024) <= 228 * 1024, "3 CTAs per SM");
   static_assert(kStages % kConsumerWarps == 0, "each stage belongs to one consumer warp");
   static_assert(CHUNKED || kMergeBytes <= kRingBytes, "merge buffer fits the idle ring");
 };
@@ -135,10 +140,9 @@ struct DecodeParams {
   int max_partitions;           // P (workspace stride)
   float score_scale;            // sm_scale * log2(e) [* k_scale for fp8]
   float out_scale;              // v_scale for fp8, 1 for bf16
-  // fused write of the step's new token (append != 0): sequence s's new K
-  // and V rows (bf16 [S][Hkv][D]) go to slot L_s - 1 of its table before
-  // anything reads that block
-  int append;
+  // fused write of the step's new token (the APPEND instantiations):
+  // sequence s's new K and V rows (bf16 [S][Hkv][D]) go to slot L_s - 1 of
+  // its table
   const uint16_t *new_k;
   const uint16_t *new_v;
   void *k_cache;
@@ -500,11 +504,12 @@ __device__ __forceinline__ void merge_and_write(WarpState<D, NT> &ws, float *mbu
   }
 }
 
-template <int D, bool FP8, int NT, bool CHUNKED>
-__global__ void __launch_bounds__(kDecodeThreads)
-    paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_v,
-                        const DecodeParams p) {
+// The kernel body; paged_decode_kernel (one head tile) and
+// paged_decode_kernel_wide (two head tiles, groups of 9-16 query heads)
+// below launch it.
+template <int D, bool FP8, int NT, bool CHUNKED, bool APPEND>
+__device__ __forceinline__ void decode_body(const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
+                                            const DecodeParams &p) {
   using G = Geo<D, FP8>;
   using PL = Plan<D, FP8, NT, CHUNKED>;
   constexpr int NS = PL::kStages;
@@ -564,32 +569,30 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
     const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
     // Fused write of the step's new token (pa_decode_append): the CTA whose
-    // range holds the token's block writes the token's K and V rows of this
-    // KV head (one 8-element chunk per lane). The rows are loaded at once,
-    // stored once the first stage's loads are issued (so their latency does
-    // not hold up the stream), and fenced against the TMA reads right before
-    // the load of the token's block. An id outside the pool is left alone
-    // (its loads read zeros and are flagged below).
-    int write_stage = -1;  // ring stage holding the new token's block
+    // range holds the token's block stores the token's K and V rows of this
+    // KV head to the cache (one 8-element chunk per lane) after issuing all
+    // its loads, so that fetching the row never holds up the stream.
+    // Nothing in this launch reads those bytes back through TMA: the row
+    // also goes to a shared slot before the arrive on its stage's full
+    // barrier (which releases it), and the consumer that attends that
+    // block patches it into its staged tile. An id outside the pool is left
+    // alone (its loads read zeros and are flagged below).
     bool pending = false;  // this lane has a chunk to store
     uint4 new_kx = make_uint4(0u, 0u, 0u, 0u), new_vx = new_kx;
     int64_t new_dst = 0;
-    if (p.append && L > 0 && !bad_len) {
+    int new_stage = -1, new_blk = 0;
+    if (APPEND && L > 0 && !bad_len) {
       const int jl = (L - 1) / kBS;
       if (jl >= j0 && jl < j1) {
-        write_stage = (jl - j0) / BPS;
-        const int pid = bt[jl];
-        if (lane < D / 8 && pid >= 0 && pid < p.num_blocks) {
+        new_stage = (jl - j0) / BPS;
+        new_blk = (jl - j0) % BPS;
+        if (lane < D / 8) {  // in flight until that stage comes round
           const int64_t src = (static_cast<int64_t>(s) * p.num_kv_heads + h) * D + lane * 8;
           new_kx = *reinterpret_cast<const uint4 *>(p.new_k + src);
           new_vx = *reinterpret_cast<const uint4 *>(p.new_v + src);
-          new_dst = ((static_cast<int64_t>(pid) * p.num_kv_heads + h) * kBS + (L - 1) % kBS) * D +
-                    lane * 8;
-          pending = true;
         }
       }
     }
-    bool stored = false;
     int issued = 0;
     bool ok = true;
     bool bad_id = false;
@@ -602,14 +605,22 @@ __global__ void __launch_bounds__(kDecodeThreads)
         int phys[BPS];
 #pragma unroll
         for (int b = 0; b < BPS; ++b) phys[b] = __shfl_sync(0xffffffffu, mine, i * BPS + b - jb);
-        if (pending && !stored && (i > 0 || i == write_stage)) {
-          store_kv_chunk<FP8>(new_kx, new_vx, p.k_cache, p.v_cache, new_dst, p.k_scale,
-                              p.v_scale);
-          stored = true;
-        }
-        if (i == write_stage) {  // the new token's row is stored before its block is read
-          if (stored) fence_proxy_async_global();
-          __syncwarp();
+        if (i == new_stage) {
+          int pid = -1;  // the block id, from the window already in hand
+#pragma unroll
+          for (int b = 0; b < BPS; ++b)
+            if (b == new_blk) pid = phys[b];
+          const bool in_pool = pid >= 0 && pid < p.num_blocks;
+          uint4 *slot = reinterpret_cast<uint4 *>(base_ptr + PL::kPatchOffset);
+          if (lane < D / 8) {
+            slot[lane] = new_kx;
+            slot[D / 8 + lane] = new_vx;
+            pending = in_pool;
+            new_dst = ((static_cast<int64_t>(pid) * p.num_kv_heads + h) * kBS + (L - 1) % kBS) * D +
+                      lane * 8;
+          }
+          if (lane == 0) *reinterpret_cast<int *>(slot + D / 4) = in_pool;
+          __syncwarp();  // ordered before lane 0's arrive below
         }
         if (lane == 0) {
           const int st = i % NS;
@@ -652,6 +663,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         if (!ok) break;
       }
     }
+    if (pending)  // after every load is issued: nothing here waits on this
+      store_kv_chunk<FP8>(new_kx, new_vx, p.k_cache, p.v_cache, new_dst, p.k_scale, p.v_scale);
     if (lane == 0) {
       if (bad_id) raise_error(kErrBlockRange);
       // No bulk copy may still be landing in this CTA's shared memory when
@@ -722,6 +735,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
   }
 
+  // pa_decode_append: the stage, block and row of the new token, if this
+  // CTA streams its (valid) block; that stage's consumer patches the row.
+  int patch_stage = -1, patch_blk = 0;
+  if (APPEND && L > 0 && !bad_len) {
+    const int jl = (L - 1) / kBS;
+    if (jl >= j0 && jl < j1) {
+      patch_stage = (jl - j0) / BPS;
+      patch_blk = (jl - j0) % BPS;
+    }
+  }
+
   // Stages of this warp: i = warp, warp + 4, ... over [0, nst). In a split
   // chunk every partition is a whole number of rounds (pb / BPS stages, a
   // multiple of 4), so all warps cross a partition boundary together.
@@ -749,6 +773,27 @@ __global__ void __launch_bounds__(kDecodeThreads)
         kt[b] = k0 + b * G::kTileBytes;
         vt[b] = k0 + (BPS + b) * G::kTileBytes;
       }
+      if (i == patch_stage) {
+        // the new token's row: the staged copy may predate the store, so
+        // write the row into the tile (same bytes as the cache store)
+        const int r = (L - 1) % kBS;
+        // written by the producer before its arrive on this stage
+        const uint4 *slot = reinterpret_cast<const uint4 *>(base_ptr + PL::kPatchOffset);
+        if (lane < D / 8 && *reinterpret_cast<const int *>(slot + D / 4) != 0) {
+          const uint4 patch_k = slot[lane];
+          const uint4 patch_v = slot[D / 8 + lane];
+          if constexpr (!FP8) {
+            st_shared_v4(kt[patch_blk] + swz<D, FP8>(r, lane * 16), patch_k);
+            st_shared_v4(vt[patch_blk] + swz<D, FP8>(r, lane * 16), patch_v);
+          } else {
+            st_shared_v2(kt[patch_blk] + swz<D, FP8>(r, lane * 8), e4m3_chunk(patch_k, p.k_scale));
+            st_shared_v2(vt[patch_blk] + swz<D, FP8>(r, lane * 8), e4m3_chunk(patch_v, p.v_scale));
+          }
+          // the stage is refilled by TMA later: order these writes first
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+      }
       const int valid = tok_end - (j0 + i * BPS) * kBS;  // real tokens in this stage
       if (valid >= BPS * kBS)
         attend_blocks<D, FP8, NT, BPS, false>(kt, vt, BPS * kBS, lane, qf, cs, ws);
@@ -767,6 +812,24 @@ __global__ void __launch_bounds__(kDecodeThreads)
                                   false);
     }
   }
+}
+
+// APPEND is a separate instantiation so that the plain decode carries none
+// of the fused write's code.
+template <int D, bool FP8, bool CHUNKED, bool APPEND>
+__global__ void __launch_bounds__(kDecodeThreads)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  decode_body<D, FP8, 1, CHUNKED, APPEND>(tmap_k, tmap_v, p);
+}
+
+// Two head tiles hold ~110 registers of state per thread; the cap keeps two
+// CTAs per SM (200 x 160 x 2 registers).
+template <int D, bool FP8, bool CHUNKED, bool APPEND>
+__global__ void __maxnreg__(200)
+    paged_decode_kernel_wide(const __grid_constant__ CUtensorMap tmap_k,
+                             const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  decode_body<D, FP8, 2, CHUNKED, APPEND>(tmap_k, tmap_v, p);
 }
 
 // Combine the partitions of one (sequence, query head):

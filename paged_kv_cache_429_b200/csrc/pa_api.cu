@@ -106,7 +106,7 @@ bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int 
   return true;
 }
 
-template <int D, bool FP8, int NT, bool CHUNKED>
+template <int D, bool FP8, int NT, bool CHUNKED, bool APPEND>
 pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
                         const DecodeParams &p, int num_seqs, int grid_x,
                         cudaStream_t stream, int dev) {
@@ -114,7 +114,8 @@ pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
   if (!make_cache_tmap<D, FP8>(&tk, k_cache, rows) ||
       !make_cache_tmap<D, FP8>(&tv, v_cache, rows))
     return PA_ERR_CUDA;
-  auto kern = pa::paged_decode_kernel<D, FP8, NT, CHUNKED>;
+  auto kern = NT == 1 ? pa::paged_decode_kernel<D, FP8, CHUNKED, APPEND>
+                      : pa::paged_decode_kernel_wide<D, FP8, CHUNKED, APPEND>;
   static std::atomic<uint64_t> attr_done{0};
   const size_t smem = pa::Plan<D, FP8, NT, CHUNKED>::kSmemBytes;
   if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
@@ -134,11 +135,18 @@ template <int D, bool FP8>
 pa_status dispatch_nt(int nt, bool chunked, const void *kc, const void *vc, int rows,
                       const DecodeParams &p, int num_seqs, int grid_x, cudaStream_t st,
                       int dev) {
+  if (p.new_k) {
+    if (chunked)
+      return nt == 1 ? launch_decode<D, FP8, 1, true, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                     : launch_decode<D, FP8, 2, true, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+    return nt == 1 ? launch_decode<D, FP8, 1, false, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                   : launch_decode<D, FP8, 2, false, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+  }
   if (chunked)
-    return nt == 1 ? launch_decode<D, FP8, 1, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
-                   : launch_decode<D, FP8, 2, true>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
-  return nt == 1 ? launch_decode<D, FP8, 1, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
-                 : launch_decode<D, FP8, 2, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+    return nt == 1 ? launch_decode<D, FP8, 1, true, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                   : launch_decode<D, FP8, 2, true, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
+  return nt == 1 ? launch_decode<D, FP8, 1, false, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev)
+                 : launch_decode<D, FP8, 2, false, false>(kc, vc, rows, p, num_seqs, grid_x, st, dev);
 }
 
 // Consecutive partitions per CTA in the split path: about 1 MB of K/V per
@@ -273,8 +281,7 @@ static pa_status decode_common(float *out, const void *q, const void *k_cache,
   p.num_kv_heads = num_kv_heads;
   p.group = group;
   p.num_blocks = num_blocks;
-  if (new_k) {
-    p.append = 1;
+  if (new_k) {  // selects the APPEND kernels
     p.new_k = static_cast<const uint16_t *>(new_k);
     p.new_v = static_cast<const uint16_t *>(new_v);
     p.k_cache = const_cast<void *>(k_cache);
