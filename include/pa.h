@@ -140,12 +140,14 @@ PA_API pa_status pa_decode(float *out, const void *q, const void *k_cache,
  * block_tables[s][(L - 1) / 16] * 16 + (L - 1) % 16 of the caches exactly
  * as pa_reshape_and_cache would (bf16 bits, or E4M3(x / scale) with the
  * given k_scale / v_scale), then computes the same output as pa_decode —
- * in the decode launch itself, which writes the token before it reads that
- * block ([Ch7] §7.1 "Block 与 Block Table": a generated token goes into the
- * next slot of the sequence's last block). The pages have no separate call
- * for this; it saves the cache-write launch of every decode step. Any
- * copy-on-write copy of a shared last block (pa_copy_blocks) must come
- * first.
+ * in the decode launch itself: the CTA that streams the sequence's last
+ * block stores the row and attends to the same row, so caches and output
+ * are bit-identical to pa_reshape_and_cache followed by pa_decode ([Ch7]
+ * §7.1 "Block 与 Block Table": a generated token goes into the next slot
+ * of the sequence's last block). The pages have no separate call for this;
+ * it saves the cache-write launch of every decode step, which matters
+ * where a step is launch-bound. Any copy-on-write copy of a shared last
+ * block (pa_copy_blocks) must come first.
  *   key, value   bf16 [num_seqs][num_kv_heads][head_dim], 16-byte aligned.
  *   k_cache, v_cache  written in place (the new slots only).
  *   Other arguments as for pa_decode. A table entry outside the pool is
