@@ -177,6 +177,12 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def quantiles_ms(xs, fracs=(0.1, 0.5, 0.9)):
+    """Nearest-rank quantiles of a list of durations, rounded to ns."""
+    s = sorted(xs)
+    return [round(s[min(len(s) - 1, int(f * (len(s) - 1) + 0.5))], 6) for f in fracs]
+
+
 def init_dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -337,7 +343,9 @@ def run_ours(args, world, rank, local):
                      "kernel": "paged_decode_kernel" + (" (new-token write fused)" if fuse else "")
                                + (" + reduce" if split else ""),
                      "algorithmic_bytes_per_launch": kernel_bytes,
-                     "avg_launch_ms": round(dec_avg_ms, 6), "peak_source": peak_src},
+                     "avg_launch_ms": round(dec_avg_ms, 6),
+                     "launch_ms_p10_p50_p90": quantiles_ms(dec_ms),
+                     "launches_timed": len(dec_ms), "peak_source": peak_src},
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
