@@ -203,7 +203,7 @@ class DecodeBatch:
                    workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         """The same step with the new tokens' write fused into the decode
         launch (pa_decode_append): any copy-on-write copies first, then one
-        decode that writes each sequence's new token before reading it."""
+        decode that also writes each sequence's new token and attends to it."""
         writes = [op for op in self.step_ops if op.kind == "write"]
         assert len(writes) == 1 and writes[0].src == "new" and writes[0].row0 == 0 \
             and writes[0].row1 == self.w.num_seqs
