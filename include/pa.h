@@ -85,7 +85,9 @@ PA_API const char *pa_status_string(pa_status status);
  * the automatic choice (sized for its split default, 512 tokens); 0 means
  * single-pass, which needs no workspace (returns 0). The size is
  * num_seqs * num_q_heads * ceil(max_context_len / partition) * (head_dim+2)
- * floats, rounded up to 256 bytes. Returns 0 for invalid arguments. */
+ * floats plus 512 bytes (the partial outputs and the (max, sum) pairs each
+ * start 256-byte aligned), rounded up to 256 bytes. Returns 0 for invalid
+ * arguments. */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim,
                                 int max_context_len, int partition_size);
 
