@@ -272,6 +272,18 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize(device)
+    run_step = one_step
+    if args.graph:
+        # the whole step captured once (on torch's capture stream) and
+        # replayed on this stream: no host work per step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            one_step()
+        torch.cuda.synchronize(device)
+        run_step = graph.replay
+        for _ in range(args.warmup):
+            run_step()
+        torch.cuda.synchronize(device)
 
     # ---- device-resident timing: K whole steps, nothing else on the stream
     K = args.steps
@@ -282,7 +294,7 @@ def run_ours(args, world, rank, local):
     clocks.start()
     t0.record(stream)
     for i in range(K):
-        one_step()
+        run_step()
     t1.record(stream)
     torch.cuda.synchronize(device)
     clocks.stop()
@@ -325,6 +337,7 @@ def run_ours(args, world, rank, local):
             "new_token_write": "fused into the decode launch (pa_decode_append)" if fuse
                                else "separate pa_reshape_and_cache launch",
             "partition_size": ps,
+            "step_launch": "one CUDA graph replay" if args.graph else "eager calls",
             "l2": (f"inputs larger than L2: {decode_bytes / 1e9:.2f} GB per step vs "
                    f"{L2_BYTES / 2**20:.0f} MiB L2; no flush"),
             "seed": args.seed,
@@ -688,6 +701,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--fuse", action="store_true",
                     help="write the new tokens inside the decode launch (pa_decode_append) "
                          "instead of a separate pa_reshape_and_cache launch")
