@@ -22,7 +22,10 @@
  *     says "host". The library allocates no memory of its own.
  *   - GPU work is launched asynchronously on `stream` (a cudaStream_t;
  *     NULL is the legacy default stream). No call synchronises, except
- *     pa_get_device_error.
+ *     pa_get_device_error. The launching calls can therefore be captured
+ *     in a CUDA graph and replayed (pa_decode_no_alloc once it has been
+ *     called on the device outside a capture); the split path's workspace
+ *     must then stay allocated for the graph's lifetime.
  *   - Arguments are checked on the host before anything is launched; on a
  *     non-OK status nothing was launched. A failed launch returns
  *     PA_ERR_CUDA.
