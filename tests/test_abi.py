@@ -180,3 +180,26 @@ def test_binding_argument_counts_match_the_header():
     arity = declared_arity()
     for name, (_, args) in _lib.SIGNATURES.items():
         assert len(args) == arity[name], (name, len(args), arity[name])
+
+
+def test_product_never_reaches_the_oracle():
+    """The oracle is test infrastructure: no module of the package imports
+    it and no CUDA/C++ source includes anything from it."""
+    import ast
+    pkg = os.path.dirname(_lib.LIB_PATH)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                tree = ast.parse(open(path, encoding="utf-8").read(), path)
+                for node in ast.walk(tree):
+                    if isinstance(node, ast.Import):
+                        names = [a.name for a in node.names]
+                    elif isinstance(node, ast.ImportFrom):
+                        names = [node.module or ""]
+                    else:
+                        continue
+                    assert not any(n.split(".")[0] == "oracle" for n in names), (path, names)
+            elif f.endswith((".cu", ".cuh", ".cpp", ".h")):
+                src = open(path, encoding="utf-8").read()
+                assert not re.search(r'#\s*include\s*[<"][^>"]*oracle', src), path
