@@ -203,3 +203,30 @@ def test_product_never_reaches_the_oracle():
             elif f.endswith((".cu", ".cuh", ".cpp", ".h")):
                 src = open(path, encoding="utf-8").read()
                 assert not re.search(r'#\s*include\s*[<"][^>"]*oracle', src), path
+
+
+def test_oracle_never_reaches_the_product():
+    """The oracle shares no code with the CUDA path: it neither imports the
+    package nor includes its headers or sources."""
+    import ast
+    root = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle")
+    for dirpath, _, files in os.walk(root):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                tree = ast.parse(open(path, encoding="utf-8").read(), path)
+                for node in ast.walk(tree):
+                    if isinstance(node, ast.Import):
+                        names = [a.name for a in node.names]
+                    elif isinstance(node, ast.ImportFrom):
+                        names = [node.module or ""]
+                    else:
+                        continue
+                    assert not any(n.split(".")[0] == "paged_kv_cache_429_b200" for n in names), \
+                        (path, names)
+            elif f.endswith((".c", ".h", ".cpp")):
+                src = open(path, encoding="utf-8").read()
+                for inc in re.findall(r'#\s*include\s*[<"]([^>"]+)[>"]', src):
+                    assert inc in {"stdint.h", "stddef.h", "stdlib.h", "string.h", "math.h",
+                                   "stdio.h", "float.h", "limits.h"} or inc.startswith("oracle"), \
+                        (path, inc)
