@@ -1,5 +1,10 @@
 """Host-side helpers of bench.py: launch-time quantiles and the gating of the
-ncu traffic figure on the decode source it was captured from."""
+ncu traffic figure on the decode source it was captured from; the CPU
+oracle arm (--impl reference) and its JSON line."""
+import json
+
+import pytest
+
 import bench
 
 
@@ -35,3 +40,39 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("stale") is None
     assert bench.profiled_traffic("nohash") is None
     assert bench.profiled_traffic("missing") is None
+
+
+def _run_main(argv, capsys, monkeypatch, env=None):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    for k, v in (env or {}).items():
+        monkeypatch.setenv(k, v)
+    bench.main(argv)
+    return [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    """--impl reference times the CPU oracle and prints the contract's line."""
+    lines = _run_main(["--impl", "reference", "--steps", "3", "--warmup", "3"], capsys,
+                      monkeypatch)
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s"
+    assert d["steps"] == 3 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["higher_is_better"] is True and d["gpu_launches"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("llama7b")
+
+
+def test_reference_arm_other_ranks_print_nothing(capsys, monkeypatch):
+    lines = _run_main(["--impl", "reference", "--steps", "3", "--warmup", "3"], capsys,
+                      monkeypatch, env={"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"})
+    assert lines == []
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--steps", "3", "--warmup", "2"])
