@@ -411,6 +411,10 @@ PA_API int pa_pool_num_free(const pa_pool *pool);
 PA_API int pa_pool_refcount(const pa_pool *pool, int block_id); /* -1 if invalid   */
 /* Length (tokens) and block count of a sequence; -1 if unknown. */
 PA_API int64_t pa_pool_seq_len(const pa_pool *pool, int64_t seq_id);
+/* The lengths of n sequences at once (int64 [n], host; -1 for an unknown
+ * id): one call per scheduling step instead of one per sequence. */
+PA_API pa_status pa_pool_seq_lens(const pa_pool *pool, const int64_t *seq_ids, int n,
+                                  int64_t *lens_out);
 PA_API int pa_pool_seq_num_blocks(const pa_pool *pool, int64_t seq_id);
 
 #ifdef __cplusplus

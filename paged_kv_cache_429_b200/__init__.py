@@ -416,5 +416,14 @@ class BlockPool:
     def seq_len(self, seq_id: int) -> int:
         return int(self._lib.pa_pool_seq_len(self._h, seq_id))
 
+    def seq_lens(self, seq_ids) -> np.ndarray:
+        """Lengths of many sequences in one call (-1 for an unknown id)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty(len(ids), dtype=np.int64)
+        n = len(ids)
+        _ok(self._lib.pa_pool_seq_lens(self._h, ids.ctypes.data if n else None, n,
+                                       out.ctypes.data if n else None), "pa_pool_seq_lens")
+        return out
+
     def seq_num_blocks(self, seq_id: int) -> int:
         return int(self._lib.pa_pool_seq_num_blocks(self._h, seq_id))

@@ -57,6 +57,7 @@ SIGNATURES = {
     "pa_pool_num_free": (_i32, [_vp]),
     "pa_pool_refcount": (_i32, [_vp, _i32]),
     "pa_pool_seq_len": (_i64, [_vp, _i64]),
+    "pa_pool_seq_lens": (_i32, [_vp, _vp, _i32, _vp]),
     "pa_pool_seq_num_blocks": (_i32, [_vp, _i64]),
 }
 

@@ -456,6 +456,16 @@ int64_t pa_pool_seq_len(const pa_pool *pool, int64_t seq_id) {
   return it == pool->seqs.end() ? -1 : it->second.len;
 }
 
+pa_status pa_pool_seq_lens(const pa_pool *pool, const int64_t *seq_ids, int n,
+                           int64_t *lens_out) {
+  if (!pool || n < 0 || (n > 0 && (!seq_ids || !lens_out))) return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    auto it = pool->seqs.find(seq_ids[i]);
+    lens_out[i] = it == pool->seqs.end() ? -1 : it->second.len;
+  }
+  return PA_OK;
+}
+
 int pa_pool_seq_num_blocks(const pa_pool *pool, int64_t seq_id) {
   if (!pool) return -1;
   auto it = pool->seqs.find(seq_id);

@@ -183,25 +183,23 @@ class DecodeLoop:
         # a new block needs one from the pool: preempt (swap out) the most
         # recently admitted requests until the pool covers them all.
         while True:
-            need = sum(1 for r in self.running if self.pool.seq_len(r.rid) % BS == 0)
+            cur = self.pool.seq_lens([r.rid for r in self.running])  # one call
+            need = int(np.count_nonzero(cur % BS == 0))
             if need <= self.pool.num_free or not self.running:
                 break
             if not self._preempt(keep=None):
                 raise RuntimeError("out of GPU blocks and of swap space")
-        new_slots = {}
-        if self.running:
-            ids = np.array([r.rid for r in self.running], dtype=np.int64)
+        # every running request gets its slot (in order) or the call raises
+        batch = list(self.running)
+        n = len(batch)
+        if n:
+            ids = np.fromiter((r.rid for r in batch), dtype=np.int64, count=n)
             slots, cow = self.pool.append_decode(ids)
             assert len(cow) == 0  # the loop never forks, so nothing is shared
-            new_slots = dict(zip(ids.tolist(), slots.tolist()))
-        batch = [r for r in self.running if r.rid in new_slots]
-        n = len(batch)
         stats = {"step": self.step_no, "running": n, "waiting": len(self.waiting),
                  "swapped": len(self.swapped)}
         if n:
-            ids = np.array([r.rid for r in batch], dtype=np.int64)
             tables, lens = self.pool.block_tables(ids, self.width)
-            slots = np.array([new_slots[r.rid] for r in batch], dtype=np.int64)
             kv_shape = (n, c.num_kv_heads, c.head_dim)
             self._write(self._randn(kv_shape), self._randn(kv_shape), slots)
             q = self._randn((n, c.num_q_heads, c.head_dim))
@@ -213,7 +211,7 @@ class DecodeLoop:
                       self.sm_scale, workspace=self.ws)
             for r in batch:
                 r.generated += 1
-            held = int(sum(-(-int(L) // BS) for L in lens))
+            held = int(((lens.astype(np.int64) + BS - 1) // BS).sum())
             stats.update(tokens=int(lens.sum()), blocks_held=held,
                          paged_util=float(lens.sum()) / (BS * held),
                          reserved_util=float(lens.sum()) / (n * c.max_model_len),

@@ -396,3 +396,16 @@ def test_append_decode_one_token_each():
     with pytest.raises(PagedAttentionError) as e:
         small.append_decode([0])
     assert e.value.status == 5 and small.seq_len(0) == 16
+
+
+def test_seq_lens_matches_the_per_sequence_query():
+    pool = BlockPool(64)
+    for sid, n in ((5, 1), (9, 16), (2, 33)):
+        pool.add_seq(sid)
+        pool.append(sid, n)
+    pool.fork(9, 11)
+    ids = np.array([2, 11, 9, 5, 404], dtype=np.int64)
+    lens = pool.seq_lens(ids)
+    assert lens.tolist() == [33, 16, 16, 1, -1]
+    assert lens.tolist() == [pool.seq_len(int(i)) for i in ids]
+    assert pool.seq_lens(np.array([], dtype=np.int64)).tolist() == []
