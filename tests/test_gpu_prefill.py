@@ -5,7 +5,6 @@ slot first set to NaN), then prefills the last n_s tokens of each sequence:
 whole prompts (n = L), chunks after a cached prefix (n < L), and one-token
 chunks (= decode).
 """
-import dataclasses
 
 import numpy as np
 import pytest

@@ -9,7 +9,6 @@ tokens, the last-block waste bound of "GPU 学习日报 Day 28" §4.1 holds, and
 the utilisation figures are consistent; over the run, requests are
 preempted and resumed and finish, and the run is deterministic.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -7,7 +7,6 @@ the slowest rank's, its bytes the sum over ranks.
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
