@@ -277,6 +277,22 @@ def test_split_form_equals_single_pass(psize):
     np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("psize", [16, 48, 512])
+def test_split_form_equals_single_pass_fp8_gqa(psize):
+    """The same identity on E4M3 caches (per-tensor scales) with GQA groups
+    of 4: the partition + reduce form reaches the single-pass result."""
+    rng = np.random.default_rng(17)
+    lens = [1, 16, 31, 97, 700, 0]
+    q, kc, vc, bt, lens = make_case(rng, 6, 8, 2, 128, lens, 120)
+    k8 = oracle.quantize_bf16_array(kc, 0.01)
+    v8 = oracle.quantize_bf16_array(vc, 0.02)
+    kw = dict(kv_dtype=oracle.KV_FP8_E4M3, k_scale=0.01, v_scale=0.02)
+    a = oracle.paged_decode(q, k8, v8, bt, lens, 128 ** -0.5, **kw)
+    b = oracle.paged_decode_split(q, k8, v8, bt, lens, 128 ** -0.5, psize, **kw)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    assert np.all(a[5] == 0)  # empty context
+
+
 def test_seq_subset_matches_full():
     rng = np.random.default_rng(15)
     q, kc, vc, bt, lens = make_case(rng, 5, 2, 2, 64, [5, 40, 18, 2, 33], 20)
