@@ -418,6 +418,30 @@ def test_copy_blocks_copies_whole_blocks():
         oracle.copy_blocks(kc, vc, np.array([[1, 6]]))
 
 
+def test_swap_blocks_moves_blocks_between_pools():
+    """(src, dst) pairs move whole K and V blocks between a 5-block device
+    pool and an 8-block host pool and back; nothing else is touched."""
+    rng = np.random.default_rng(20)
+    gk = rng.integers(0, 65535, size=(5, 2, 16, 64)).astype(np.uint16)
+    gv = rng.integers(0, 65535, size=(5, 2, 16, 64)).astype(np.uint16)
+    hk = np.zeros((8, 2, 16, 64), dtype=np.uint16)
+    hv = hk.copy()
+    oracle.swap_blocks(hk, hv, gk, gv, np.array([[4, 7], [0, 2]]))
+    np.testing.assert_array_equal(hk[7], gk[4])
+    np.testing.assert_array_equal(hv[2], gv[0])
+    for b in (0, 1, 3, 4, 5, 6):
+        assert not hk[b].any() and not hv[b].any()
+    bk, bv = np.zeros_like(gk), np.zeros_like(gv)
+    oracle.swap_blocks(bk, bv, hk, hv, np.array([[7, 1], [2, 3]]))
+    np.testing.assert_array_equal(bk[1], gk[4])
+    np.testing.assert_array_equal(bv[3], gv[0])
+    assert not bk[[0, 2, 4]].any() and not bv[[0, 2, 4]].any()
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(hk, hv, gk, gv, np.array([[5, 0]]))  # src past the pool
+    with pytest.raises(ValueError):
+        oracle.swap_blocks(hk, hv, gk, gv, np.array([[0, 8]]))  # dst past the pool
+
+
 def test_reshape_bf16_copies_bits_and_skips_negative_slots():
     rng = np.random.default_rng(19)
     key = rng.integers(0, 65535, size=(3, 2, 64)).astype(np.uint16)
