@@ -15,6 +15,12 @@ def test_quantiles_are_nearest_rank():
     assert bench.quantiles_ms([1.0, 3.0]) == [1.0, 3.0, 3.0]
 
 
+def test_l2_note_says_which_side_of_l2_the_step_is():
+    assert bench.l2_note(1_354_125_840).startswith("inputs larger than L2: 1.35 GB")
+    small = bench.l2_note(1_050_000)
+    assert small.startswith("inputs fit in L2") and "not an HBM bandwidth figure" in small
+
+
 def test_code_only_ignores_comments_and_blank_lines():
     a = "int x = 1;  // one\n\n/* block\n comment */ int y = 2;\n"
     b = "int x = 1;\n   int y = 2;   \n"
