@@ -14,6 +14,12 @@ same metric with the step's inputs copied from pinned host memory and the
 output copied back, every step; `roofline` is the decode kernel alone.
 
   python bench.py [--gpus N --steps K --warmup W --workload NAME --impl ours|reference]
+                  [--fuse] [--graph] [--partition-size P] [--op step|loop|swap|prefill]
+
+--fuse writes the new tokens inside the decode launch (pa_decode_append);
+--graph captures one step as a CUDA graph and times its replays; --op
+selects the continuous-batching loop, block swapping or chunked prefill,
+each with its own line. --impl reference times the CPU oracle instead.
 
 With torchrun (N > 1) every rank decodes its own batch (its own sequences,
 its own pool; no collective on the data path): weak scaling.
