@@ -569,3 +569,92 @@ def test_prefill_chunks_compose():
     first = oracle.paged_prefill(q[:50], kc, vc, bt, np.array([0, 50]), [50], 0.125)
     second = oracle.paged_prefill(q[50:], kc, vc, bt, np.array([0, 40]), [90], 0.125)
     np.testing.assert_array_equal(np.concatenate([first, second]), whole)
+
+
+# ------------------------------------------------ block-table invariants
+#
+# The checker is the judge of the host pool, so each invariant it enforces is
+# pinned here by a hand-built table that breaks exactly that invariant. The
+# passing control is [Day28] §六's scenario written out by hand: request A
+# holds 20 tokens in blocks [7, 1], request B forked from it shares both
+# (refcount 2), then B's write into the partly filled block 1 copies it to
+# block 3 (A keeps [7, 1], B gets [7, 3]; block 1's refcount drops to 1).
+
+DAY28_ROWS = [[7, 1], [7, 3]]
+DAY28_LENS = [20, 21]
+DAY28_NB = 10
+DAY28_REFC = [0] * DAY28_NB
+DAY28_REFC[7], DAY28_REFC[1], DAY28_REFC[3] = 2, 1, 1
+
+
+def day28_check(rows=None, lens=None, refc=None, num_free=None, nb=DAY28_NB):
+    return oracle.check_block_tables(
+        DAY28_ROWS if rows is None else rows, DAY28_LENS if lens is None else lens,
+        nb, 16, refcounts=DAY28_REFC if refc is None else refc,
+        num_free=DAY28_NB - 3 if num_free is None else num_free)
+
+
+def test_block_table_checker_accepts_the_day28_scenario():
+    assert day28_check() == []
+    # the [7, 1, 3] table of [Day28] §3.1 alone, 48 tokens (no waste) and 33
+    # tokens (15 unused slots, the largest waste the bound allows)
+    for L in (33, 48):
+        assert oracle.check_block_tables([[7, 1, 3]], [L], 10, 16) == []
+
+
+def test_block_table_checker_reports_one_block_too_many():
+    """ceil(L/16) + 1 blocks: a whole unused block, 16 unused slots."""
+    errs = oracle.check_block_tables([[7, 1, 3]], [32], 10, 16)
+    assert any("3 blocks for 32 tokens, expected 2" in e for e in errs)
+    assert any("16 unused slots" in e for e in errs)
+    assert len(errs) == 2
+
+
+def test_block_table_checker_reports_one_block_too_few():
+    errs = oracle.check_block_tables([[7, 1]], [33], 10, 16)
+    assert any("2 blocks for 33 tokens, expected 3" in e for e in errs)
+    assert any("-1 unused slots" in e for e in errs)
+    assert len(errs) == 2
+
+
+def test_block_table_checker_waste_bound_is_fifteen_slots():
+    """The bound itself, one slot on either side of it: 15 unused slots pass
+    ([Day28] §4.2, FAQ Q2); the checker flags a waste of 16 even when only
+    the waste test could catch it (the block count is checked separately)."""
+    assert oracle.check_block_tables([[5]], [1], 10, 16) == []
+    errs = oracle.check_block_tables([[5, 6]], [16], 10, 16)
+    assert [e for e in errs if "unused slots" in e] == ["seq 0: 16 unused slots in its last block"]
+
+
+@pytest.mark.parametrize("bad", [-1, DAY28_NB, DAY28_NB + 7])
+def test_block_table_checker_reports_out_of_range_ids(bad):
+    rows = [[7, 1], [7, bad]]
+    refc = list(DAY28_REFC)
+    refc[3] = 0
+    errs = day28_check(rows=rows, refc=refc, num_free=DAY28_NB - 2)
+    assert errs[0] == f"seq 1: block id {bad} out of range"
+    # the id is counted as a use: conservation is off by that phantom block
+    assert errs[1:] == [f"{DAY28_NB - 2} free + 3 used != {DAY28_NB}"]
+
+
+@pytest.mark.parametrize("block,delta", [(7, +1), (7, -1), (1, +1), (3, -1), (0, +1)])
+def test_block_table_checker_reports_refcount_off_by_one(block, delta):
+    refc = list(DAY28_REFC)
+    refc[block] += delta
+    uses = DAY28_REFC[block]
+    assert day28_check(refc=refc) == [
+        f"block {block}: refcount {uses + delta} but {uses} table entries"]
+
+
+@pytest.mark.parametrize("num_free", [DAY28_NB - 4, DAY28_NB - 2, 0, DAY28_NB])
+def test_block_table_checker_reports_broken_conservation(num_free):
+    """free + distinct used blocks must be N: a leaked block (one free too
+    few) and a double-freed one (one too many) are both reported."""
+    assert day28_check(num_free=num_free) == [f"{num_free} free + 3 used != {DAY28_NB}"]
+
+
+def test_block_table_checker_counts_shared_blocks_once_for_conservation():
+    """Block 7 appears in two tables but is one physical block: the sum is
+    over distinct blocks, so 7 free + 3 used == 10 holds."""
+    assert day28_check(num_free=7) == []
+    assert day28_check(num_free=6) == ["6 free + 3 used != 10"]
