@@ -22,9 +22,9 @@
  *     says "host". The library allocates no memory of its own.
  *   - GPU work is launched asynchronously on `stream` (a cudaStream_t;
  *     NULL is the legacy default stream). No call synchronises, except
- *     pa_get_device_error. The launching calls can therefore be captured
- *     in a CUDA graph and replayed (pa_decode_no_alloc once it has been
- *     called on the device outside a capture); the split path's workspace
+ *     pa_get_device_error. pa_decode, pa_decode_append, pa_prefill,
+ *     pa_reshape_and_cache, pa_copy_blocks and pa_swap_blocks can therefore
+ *     be captured in a CUDA graph and replayed; the split path's workspace
  *     must then stay allocated for the graph's lifetime.
  *   - Arguments are checked on the host before anything is launched; on a
  *     non-OK status nothing was launched. A failed launch returns

@@ -71,6 +71,18 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> int:
     return s.cuda_stream
 
 
+def _device_of(*tensors: torch.Tensor) -> torch.device:
+    """The one CUDA device all CUDA tensors of a call live on.
+
+    The library launches on the calling thread's current device and looks up
+    per-device state (the no-alloc scratch, kernel attributes) there, so each
+    launching call makes this device current for its duration."""
+    devs = {t.device for t in tensors if t.is_cuda}
+    if len(devs) != 1:
+        raise ValueError(f"the call's CUDA tensors must share one device, got {sorted(map(str, devs))}")
+    return devs.pop()
+
+
 def _need(t: torch.Tensor, name: str, dtypes, ndim: int, cuda: bool = True):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -120,12 +132,14 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
             workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    rc = _lib.lib().pa_decode(
-        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-        kv_dtype_of(k_cache), float(k_scale), float(v_scale),
-        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
-        int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
-        int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
+    ws = () if workspace is None else (workspace,)
+    with torch.cuda.device(_device_of(out, q, k_cache, v_cache, block_tables, context_lens, *ws)):
+        rc = _lib.lib().pa_decode(
+            out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            kv_dtype_of(k_cache), float(k_scale), float(v_scale),
+            block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+            int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
+            int(partition_size), ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode")
     return out
 
@@ -162,12 +176,15 @@ def pa_decode_append(out: torch.Tensor, q: torch.Tensor, key: torch.Tensor,
             workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    rc = _lib.lib().pa_decode_append(
-        out.data_ptr(), q.data_ptr(), key.data_ptr(), value.data_ptr(), k_cache.data_ptr(),
-        v_cache.data_ptr(), kv_dtype_of(k_cache), float(k_scale), float(v_scale),
-        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
-        int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale), int(partition_size),
-        ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
+    ws = () if workspace is None else (workspace,)
+    with torch.cuda.device(_device_of(out, q, key, value, k_cache, v_cache, block_tables,
+                                      context_lens, *ws)):
+        rc = _lib.lib().pa_decode_append(
+            out.data_ptr(), q.data_ptr(), key.data_ptr(), value.data_ptr(), k_cache.data_ptr(),
+            v_cache.data_ptr(), kv_dtype_of(k_cache), float(k_scale), float(v_scale),
+            block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+            int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale), int(partition_size),
+            ws_ptr, ws_bytes, _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode_append")
     return out
 
@@ -193,12 +210,13 @@ def pa_decode_no_alloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor
         raise ValueError("shape mismatch between out, q and the caches")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables / context_lens must have num_seqs rows")
-    rc = _lib.lib().pa_decode_no_alloc(
-        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-        kv_dtype_of(k_cache), float(k_scale), float(v_scale),
-        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
-        int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
-        int(partition_size), _stream_ptr(stream, q.device))
+    with torch.cuda.device(_device_of(out, q, k_cache, v_cache, block_tables, context_lens)):
+        rc = _lib.lib().pa_decode_no_alloc(
+            out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            kv_dtype_of(k_cache), float(k_scale), float(v_scale),
+            block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+            int(max_context_len), S, Hq, Hkv, D, B, NB, float(sm_scale),
+            int(partition_size), _stream_ptr(stream, q.device))
     _ok(rc, "pa_decode_no_alloc")
     return out
 
@@ -221,12 +239,14 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     S = context_lens.shape[0]
     if tuple(out.shape) != (T, Hq, D) or Dc != D or query_start.shape[0] != S + 1:
         raise ValueError("shape mismatch between out, q, caches and query_start")
-    rc = _lib.lib().pa_prefill(
-        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-        kv_dtype_of(k_cache), block_tables.data_ptr(), block_tables.shape[1],
-        query_start.data_ptr(), context_lens.data_ptr(), int(max_query_len),
-        int(max_context_len), S, T, Hq, Hkv, D, B, NB, float(sm_scale),
-        _stream_ptr(stream, q.device))
+    with torch.cuda.device(_device_of(out, q, k_cache, v_cache, block_tables, query_start,
+                                      context_lens)):
+        rc = _lib.lib().pa_prefill(
+            out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            kv_dtype_of(k_cache), block_tables.data_ptr(), block_tables.shape[1],
+            query_start.data_ptr(), context_lens.data_ptr(), int(max_query_len),
+            int(max_context_len), S, T, Hq, Hkv, D, B, NB, float(sm_scale),
+            _stream_ptr(stream, q.device))
     _ok(rc, "pa_prefill")
     return out
 
@@ -246,10 +266,11 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor,
     NB, Hc, B, Dc = k_cache.shape
     if tuple(value.shape) != (T, Hkv, D) or (Hc, Dc) != (Hkv, D) or slot_mapping.shape[0] != T:
         raise ValueError("shape mismatch between key/value, caches and slots")
-    rc = _lib.lib().pa_reshape_and_cache(
-        key.data_ptr(), value.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-        slot_mapping.data_ptr(), T, Hkv, D, B, NB, kv_dtype_of(k_cache),
-        float(k_scale), float(v_scale), _stream_ptr(stream, key.device))
+    with torch.cuda.device(_device_of(key, value, k_cache, v_cache, slot_mapping)):
+        rc = _lib.lib().pa_reshape_and_cache(
+            key.data_ptr(), value.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            slot_mapping.data_ptr(), T, Hkv, D, B, NB, kv_dtype_of(k_cache),
+            float(k_scale), float(v_scale), _stream_ptr(stream, key.device))
     _ok(rc, "pa_reshape_and_cache")
 
 
@@ -262,9 +283,10 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor,
     _need(block_pairs, "block_pairs", (torch.int64,), 2)
     n = block_pairs.shape[0]
     block_bytes = k_cache[0].numel() * k_cache.element_size()
-    rc = _lib.lib().pa_copy_blocks(
-        k_cache.data_ptr(), v_cache.data_ptr(), block_pairs.data_ptr() if n else None,
-        n, block_bytes, k_cache.shape[0], _stream_ptr(stream, k_cache.device))
+    with torch.cuda.device(_device_of(k_cache, v_cache, block_pairs)):
+        rc = _lib.lib().pa_copy_blocks(
+            k_cache.data_ptr(), v_cache.data_ptr(), block_pairs.data_ptr() if n else None,
+            n, block_bytes, k_cache.shape[0], _stream_ptr(stream, k_cache.device))
     _ok(rc, "pa_copy_blocks")
 
 
@@ -283,11 +305,14 @@ def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor
         raise ValueError("source and destination caches differ in block geometry")
     n = block_pairs.shape[0]
     block_bytes = src_k[0].numel() * src_k.element_size()
-    dev = dst_k.device if dst_k.is_cuda else (src_k.device if src_k.is_cuda else None)
-    rc = _lib.lib().pa_swap_blocks(
-        dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(),
-        block_pairs.data_ptr() if n else None, n, block_bytes, src_k.shape[0],
-        dst_k.shape[0], _stream_ptr(stream, dev))
+    caches = (dst_k, dst_v, src_k, src_v)
+    dev = (_device_of(*caches, block_pairs) if any(t.is_cuda for t in caches)
+           else torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        rc = _lib.lib().pa_swap_blocks(
+            dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(),
+            block_pairs.data_ptr() if n else None, n, block_bytes, src_k.shape[0],
+            dst_k.shape[0], _stream_ptr(stream, dev))
     _ok(rc, "pa_swap_blocks")
 
 

@@ -38,13 +38,18 @@ std::mutex g_scratch_mu;
 // the runtime, with the device that will run the kernel current.
 pa_status scratch_on_current_device(void **addr) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();  // leave no sticky-looking error for the caller's next check
+    return PA_ERR_CUDA;
+  }
   if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_pa_noalloc_scratch) != cudaSuccess || !p)
+    if (cudaGetSymbolAddress(&p, g_pa_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
       return PA_ERR_CUDA;
+    }
     g_scratch_addr[dev] = p;
   }
   *addr = g_scratch_addr[dev];
@@ -72,14 +77,18 @@ pa_status pa_decode_no_alloc(float *out, const void *q, const void *k_cache,
   const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
                                                static_cast<int>(cap), partition_size);
   if (need > kNoAllocScratchBytes) return PA_ERR_WORKSPACE;  // beyond the fixed array
-  if (num_seqs == 0) return PA_OK;
+  // With no sequence pa_decode checks every argument and returns before it
+  // looks at the workspace, so the address lookup is skipped then and the
+  // accept/reject decision stays pa_decode's.
   void *scratch = nullptr;
-  const pa_status rc = scratch_on_current_device(&scratch);
-  if (rc != PA_OK) return rc;
+  if (num_seqs > 0) {
+    const pa_status rc = scratch_on_current_device(&scratch);
+    if (rc != PA_OK) return rc;
+  }
   return pa_decode(out, q, k_cache, v_cache, kv_dtype, k_scale, v_scale, block_tables,
                    max_blocks_per_seq, context_lens, max_context_len, num_seqs,
                    num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, sm_scale,
-                   partition_size, scratch, kNoAllocScratchBytes, stream);
+                   partition_size, scratch, scratch ? kNoAllocScratchBytes : 0, stream);
 }
 
 }  // extern "C"

@@ -88,6 +88,32 @@ def test_decode_rejects_bad_arguments_on_host(kw, expect):
     assert _lib.lib().pa_decode(*decode_args(**kw)) == expect
 
 
+def no_alloc_args(**kw):
+    a = decode_args(**kw)
+    del a[-3:-1]   # no workspace pointer or size
+    return a
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(S=0), OK),                       # empty batch: nothing to launch
+    # with no sequence the call still rejects what pa_decode rejects
+    (dict(S=0, B=32), UNSUPPORTED),
+    (dict(S=0, D=96), UNSUPPORTED),
+    (dict(S=0, Hq=12, Hkv=8), UNSUPPORTED),
+    (dict(S=0, dtype=1, ks=0.0), INVALID),
+    (dict(S=0, scale=float("nan")), INVALID),
+    (dict(S=0, NB=0), INVALID),
+    (dict(psize=0), INVALID),              # the split path is the only one
+    (dict(psize=-1), INVALID),
+    (dict(psize=100), INVALID),
+    (dict(maxctx=-1), INVALID),
+    # more scratch than the fixed array holds: 16 MiB / (64 * 8 * 130 * 4) partitions
+    (dict(S=64, maxb=1 << 20, maxctx=1 << 20), WORKSPACE),
+])
+def test_decode_no_alloc_rejects_bad_arguments_on_host(kw, expect):
+    assert _lib.lib().pa_decode_no_alloc(*no_alloc_args(**kw)) == expect
+
+
 @pytest.mark.parametrize("kw,expect", [
     (dict(T=0), OK),
     (dict(B=32), UNSUPPORTED),

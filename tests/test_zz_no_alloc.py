@@ -37,22 +37,38 @@ def call_no_alloc(b, out, partition_size, block_tables=None, max_context_len=Non
         w.sm_scale, partition_size, torch.cuda.current_stream().cuda_stream)
 
 
+def reference_decode(b, ps):
+    """pa_decode with a caller workspace whose every float is NaN, so a read
+    of anything the call did not write would show in its output."""
+    ws = b.workspace(ps)
+    assert ws.numel() <= SCRATCH_BYTES
+    ws.fill_(0xFF)   # 0xFFFFFFFF is a NaN in binary32
+    ref = torch.full_like(b.out, float("nan"))
+    pa_decode(ref, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
+              b.max_context_len, b.w.sm_scale, k_scale=b.k_scale,
+              v_scale=b.v_scale, partition_size=ps, workspace=ws)
+    return ref
+
+
 def test_two_calls_in_a_row_match_pa_decode():
-    cases = [("tiny", 0, 32), ("llama7b", 1, 512)]
-    for name, seed, ps in cases:
-        b = DecodeBatch.build(synth.WORKLOADS[name], seed)
-        b.step(partition_size=0)  # write the step's new tokens
-        ws = b.workspace(ps)
-        assert ws.numel() <= SCRATCH_BYTES
-        ref = torch.empty_like(b.out)
-        pa_decode(ref, b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens,
-                  b.max_context_len, b.w.sm_scale, k_scale=b.k_scale,
-                  v_scale=b.v_scale, partition_size=ps, workspace=ws)
+    """The shared array keeps whatever the previous call left in it, so each
+    call must read only what it wrote itself. The llama7b-shaped batch with
+    512-token partitions fills several MB of the array; the tiny batch with
+    32-token partitions (another partition count and row stride) then runs
+    twice in a row on top of it, and llama7b runs again over the tiny
+    batch's leftovers. Every result must match pa_decode run with a
+    NaN-filled caller workspace."""
+    big = DecodeBatch.build(synth.WORKLOADS["llama7b"], 1)
+    big.step(partition_size=0)  # write the step's new tokens
+    small = DecodeBatch.build(synth.WORKLOADS["tiny"], 0)
+    small.step(partition_size=0)
+    refs = {id(big): reference_decode(big, 512), id(small): reference_decode(small, 32)}
+    for b, ps in ((big, 512), (small, 32), (small, 32), (big, 512)):
         out = torch.full_like(b.out, float("nan"))
         assert call_no_alloc(b, out, ps) == 0
         torch.cuda.synchronize()
-        assert torch.all(torch.isfinite(out))
-        assert torch.max(torch.abs(out - ref)).item() <= PATH_TOL, name
+        assert torch.all(torch.isfinite(out)), b.w.name
+        assert torch.max(torch.abs(out - refs[id(b)])).item() <= PATH_TOL, b.w.name
 
 
 def test_scratch_larger_than_the_array_is_refused():
