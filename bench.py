@@ -115,7 +115,7 @@ class ClockSampler:
                0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -323,9 +323,12 @@ def run_ours(args, world, rank, local):
     KD = min(K, 500)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(KD)]
+    clocks_dec = ClockSampler(local)
+    clocks_dec.start()
     for i in range(KD):
         one_step(evs[i])
     torch.cuda.synchronize(device)
+    clocks_dec.stop()
     dec_ms = [a.elapsed_time(b) for a, b in evs]
     value = total_bytes / (max_ms * 1e-3) / 1e9
     ms_per_step = max_ms / K
@@ -373,7 +376,8 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_launch": kernel_bytes,
                      "avg_launch_ms": round(dec_avg_ms, 6),
                      "launch_ms_p10_p50_p90": quantiles_ms(dec_ms),
-                     "launches_timed": len(dec_ms), "peak_source": peak_src},
+                     "launches_timed": len(dec_ms), "peak_source": peak_src,
+                     "clocks": clocks_dec.summary()},
         "clocks": clocks.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -468,7 +472,7 @@ def run_e2e(batch, args, ps, ws, stream, device, world, step_bytes):
     for i in range(max(NSLOT, args.warmup)):
         e2e_step(i)
     torch.cuda.synchronize(device)
-    K = max(1, args.steps // 4)
+    K = max(50, args.steps)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, device)
     torch.cuda.synchronize(device)

@@ -105,3 +105,24 @@ def randn_bf16(shape, seed: int, workload: str, what: str,
     gen.manual_seed(stream_seed(seed, workload, what))
     return torch.randn(tuple(shape), generator=gen, device=dev,
                        dtype=torch.float32).to(torch.bfloat16)
+
+
+def prompt_kv_rows(token_ids, seed: int, num_kv_heads: int, head_dim: int):
+    """K and V rows (bf16 [n][num_kv_heads][head_dim]) for a request's
+    tokens, each row a function of the token ids up to and including its
+    own, as a model's K/V are: two requests whose token lists agree on a
+    prefix get identical rows on that prefix and unrelated rows after it.
+    Row i is N(0, 1) from a numpy stream keyed by (seed, a running 64-bit
+    FNV-1a hash of token_ids[:i+1]), rounded to bf16."""
+    h = 0xCBF29CE484222325
+    k = np.empty((len(token_ids), num_kv_heads * head_dim), np.float32)
+    v = np.empty_like(k)
+    for i, t in enumerate(token_ids):
+        for byte in int(t).to_bytes(4, "little", signed=True):
+            h = ((h ^ byte) * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+        g = np.random.default_rng([seed, h & 0xFFFFFFFF, h >> 32])
+        k[i] = g.standard_normal(num_kv_heads * head_dim, dtype=np.float32)
+        v[i] = g.standard_normal(num_kv_heads * head_dim, dtype=np.float32)
+    shape = (len(token_ids), num_kv_heads, head_dim)
+    return (torch.from_numpy(k).reshape(shape).to(torch.bfloat16),
+            torch.from_numpy(v).reshape(shape).to(torch.bfloat16))

@@ -59,30 +59,67 @@ def test_tiny_workload(seed):
     check_batch(b, paths=(0, 16, 64, 512, -1))
 
 
-@pytest.mark.parametrize("seed", [0, 1])
+@pytest.mark.parametrize("seed", [0, 1, 2])
 def test_llama7b_workload(seed):
     b = DecodeBatch.build(synth.WORKLOADS["llama7b"], seed)
     check_batch(b, paths=(-1, 0, 512))
 
 
-def test_prefix_workload_sampled():
-    b = DecodeBatch.build(synth.WORKLOADS["prefix"], 0)
+def sampled_subset(n, seed, must, count=32):
+    """`count` sequences of an n-sequence batch: the listed ones plus a
+    seeded draw of the rest."""
+    rest = [s for s in range(n) if s not in must]
+    pick = np.random.default_rng(100 + seed).choice(rest, count - len(must), replace=False)
+    return sorted(set(must) | set(int(x) for x in pick))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_prefix_workload_sampled(seed):
+    """32 of the 256 sequences (the first, the last writer to copy its
+    shared partial block, the last one, which writes in place, and a seeded
+    draw), all heads and dims."""
+    b = DecodeBatch.build(synth.WORKLOADS["prefix"], seed)
     assert len([op for op in b.setup_ops + b.step_ops if op.kind == "copy"]) >= 1
-    n_pairs = sum(len(op.pairs) for op in b.setup_ops + b.step_ops if op.kind == "copy")
+    copies = [op for op in b.setup_ops + b.step_ops if op.kind == "copy"]
+    n_pairs = sum(len(op.pairs) for op in copies)
     assert n_pairs == 255
-    subset = [0, 1, 77, 128, 200, 254, 255]
+    owners = set(int(o) for op in copies for o in op.owner)
+    assert owners == set(range(255))              # every writer but the last copies
+    subset = sampled_subset(256, seed, [0, 1, 254, 255])
     check_batch(b, subset, paths=(-1, 0, 512))
 
 
-def test_gqa_fp8_workload_sampled():
-    b = DecodeBatch.build(synth.WORKLOADS["gqa_fp8"], 0)
-    subset = [0, 5, 63, 64, 100, 127]
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_gqa_fp8_workload_sampled(seed):
+    b = DecodeBatch.build(synth.WORKLOADS["gqa_fp8"], seed)
+    subset = sampled_subset(128, seed, [0, 63, 64, 127])
     check_batch(b, subset, paths=(-1, 0, 512))
 
 
-def test_long_context_workload_sampled():
-    b = DecodeBatch.build(synth.WORKLOADS["long"], 0)
-    check_batch(b, [0, 5], paths=(512,))
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_long_context_workload(seed):
+    """All 8 sequences of 64K-128K tokens against the oracle: the
+    workload's own 512-token split, the automatic choice, and the step with
+    the new tokens' write fused into the decode (pa_decode_append)."""
+    b = DecodeBatch.build(synth.WORKLOADS["long"], seed)
+    kc, vc = oracle_caches(b)
+    ref = oracle_decode(b, kc, vc)
+    ws = b.workspace(512)
+    for i, ps in enumerate((512, -1)):
+        if i == 0:
+            b.step(partition_size=ps, workspace=ws)
+        else:
+            b.decode(partition_size=ps, workspace=ws)
+        torch.cuda.synchronize()
+        assert max_abs_err(b.out, ref) <= tolerance(b), ps
+    assert_cache_equal(b, kc, vc)
+    # the fused step writes the same new-token bytes again and decodes
+    b.out.fill_(float("nan"))
+    b.step_fused(partition_size=512, workspace=ws)
+    torch.cuda.synchronize()
+    assert max_abs_err(b.out, ref) <= tolerance(b), "fused"
+    assert_cache_equal(b, kc, vc)
+    assert pa_get_device_error() == 0
 
 
 # --------------------------------------------------------------- edge cases

@@ -65,3 +65,21 @@ def test_sentinels_are_nan():
     assert torch.isnan(b.view(torch.bfloat16).float()).all()
     f8 = torch.tensor([synth.SENTINEL_FP8], dtype=torch.uint8).view(torch.float8_e4m3fn)
     assert torch.isnan(f8.float()).all()
+
+
+def test_prompt_rows_depend_on_the_whole_prefix():
+    """Rows agree exactly where two token lists share a prefix and differ
+    from the first differing token on, even if later tokens agree again."""
+    a = [5, 6, 7, 8, 9]
+    b = [5, 6, 1, 8, 9]
+    ka, va = synth.prompt_kv_rows(a, 3, 2, 16)
+    kb, vb = synth.prompt_kv_rows(b, 3, 2, 16)
+    assert ka.dtype == torch.bfloat16 and ka.shape == (5, 2, 16)
+    assert torch.equal(ka[:2], kb[:2]) and torch.equal(va[:2], vb[:2])
+    for i in range(2, 5):
+        assert not torch.equal(ka[i], kb[i]) and not torch.equal(va[i], vb[i])
+    assert not torch.equal(ka, va)
+    k2, _ = synth.prompt_kv_rows(a, 4, 2, 16)     # another seed, other rows
+    assert not torch.equal(ka[0], k2[0])
+    kx, _ = synth.prompt_kv_rows(a[:3], 3, 2, 16)  # a prefix alone: same rows
+    assert torch.equal(kx, ka[:3])
