@@ -85,7 +85,8 @@ PA_API const char *pa_status_string(pa_status status);
 
 /* Bytes of workspace pa_decode needs for the split-context path.
  * partition_size: tokens per partition, a positive multiple of 16; -1 means
- * the automatic choice (sized for its split default, 512 tokens); 0 means
+ * the automatic choice (sized for the largest it can pick: 512-token
+ * partitions); 0 means
  * single-pass, which needs no workspace (returns 0). The size is
  * num_seqs * num_q_heads * ceil(max_context_len / partition) * (head_dim+2)
  * floats plus 512 bytes (the partial outputs and the (max, sum) pairs each
@@ -119,7 +120,11 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_d
  *                 host read is made). Lengths above it, above
  *                 16 * max_blocks_per_seq, or below 0 are clamped and flagged
  *                 with PA_DEVERR_CONTEXT_CLAMP.
- *   partition_size   -1 automatic; 0 forces single-pass (one CTA per
+ *   partition_size   -1 automatic: single-pass when the (sequence, KV
+ *                 head) pairs fill two waves of resident CTAs and no context
+ *                 exceeds 16384 tokens; otherwise (given a workspace) split,
+ *                 into 2048-token partitions above 16384 tokens and 512-token
+ *                 partitions below. 0 forces single-pass (one CTA per
  *                 sequence and KV head covers the whole context); a positive
  *                 multiple of 16 forces the split-context path ([Day28] §二
  *                 names the long-context "v2" kernel): each partition keeps

@@ -22,7 +22,9 @@ using pa::Geo;
 using pa::ReduceParams;
 
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultPartition = 512;
+constexpr int kDefaultPartition = 512;   // automatic split, contexts up to kLongContext
+constexpr int kLongPartition = 2048;     // automatic split above kLongContext tokens
+constexpr int kLongContext = 16384;
 
 bool aligned(const void *ptr, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
@@ -260,13 +262,16 @@ static pa_status decode_common(float *out, const void *q, const void *k_cache,
     // Single-pass when the (sequence, KV head) pairs fill at least two full
     // waves of resident CTAs (3 per SM) and contexts are not long enough for
     // the last wave's imbalance to matter; otherwise split the contexts.
+    // Above kLongContext tokens the partitions are 2048 tokens long: a
+    // quarter of the partial records to write and combine, and the grid
+    // still holds the same number of CTAs (each streams about 1 MB).
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
     const bool wide = units >= 2LL * 3 * device_sm_count(dev);
-    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap,
-                                            kDefaultPartition);
+    const int auto_ps = ctx_cap > kLongContext ? kLongPartition : kDefaultPartition;
+    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, ctx_cap, auto_ps);
     const bool have_ws = workspace && aligned(workspace, 256) && workspace_bytes >= need;
-    psize = (!wide || ctx_cap > 16384) && have_ws && ctx_cap > kDefaultPartition
-                ? kDefaultPartition
+    psize = (!wide || ctx_cap > kLongContext) && have_ws && ctx_cap > kDefaultPartition
+                ? auto_ps
                 : 0;
   }
 

@@ -60,6 +60,55 @@ class Request:
     admitted_at: int = -1
 
 
+class _Staging:
+    """Page-locked staging for the host arrays one step sends to the GPU
+    (cache slots, swap pairs, block tables, context lengths). They are
+    packed into the next buffer of a small ring and sent with one
+    non-blocking copy on the current stream, so the host never waits for
+    the GPU to drain before an upload and its scheduling of the next step
+    runs while the GPU still works on this one. A ring buffer is refilled
+    only once the copy that last read it has completed (an event recorded
+    behind that copy; with a ring of three it is long done)."""
+
+    ALIGN = 256
+
+    def __init__(self, device: torch.device, depth: int = 3, nbytes: int = 1 << 20):
+        self.device = device
+        self.depth = depth
+        self.host = [torch.empty(nbytes, dtype=torch.uint8).pin_memory() for _ in range(depth)]
+        self.dev = [torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(depth)]
+        self.events: List[Optional[torch.cuda.Event]] = [None] * depth
+        self.i = 0
+
+    def upload(self, arrays: List[np.ndarray]) -> List[torch.Tensor]:
+        k = self.i % self.depth
+        self.i += 1
+        offs, total = [], 0
+        for a in arrays:
+            offs.append(total)
+            total += -(-a.nbytes // self.ALIGN) * self.ALIGN
+        if self.events[k] is not None:
+            self.events[k].synchronize()
+        if total > self.host[k].numel():
+            n = max(total, 2 * self.host[k].numel())
+            self.host[k] = torch.empty(n, dtype=torch.uint8).pin_memory()
+            self.dev[k] = torch.empty(n, dtype=torch.uint8, device=self.device)
+        hbuf = self.host[k].numpy()
+        for a, o in zip(arrays, offs):
+            hbuf[o:o + a.nbytes] = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+        if total:
+            self.dev[k][:total].copy_(self.host[k][:total], non_blocking=True)
+        if self.device.type == "cuda":
+            ev = torch.cuda.Event()
+            ev.record()
+            self.events[k] = ev
+        return [self.dev[k][o:o + a.nbytes].view(_TORCH_DTYPE[a.dtype]).view(a.shape)
+                for a, o in zip(arrays, offs)]
+
+
+_TORCH_DTYPE = {np.dtype(np.int64): torch.int64, np.dtype(np.int32): torch.int32}
+
+
 class DecodeLoop:
     def __init__(self, cfg: LoopConfig, device="cuda", record: bool = False):
         self.cfg = cfg
@@ -92,6 +141,11 @@ class DecodeLoop:
         self.ws = torch.empty(pa_decode_workspace_size(cfg.max_num_seqs, cfg.num_q_heads,
                                                        cfg.head_dim, cfg.max_model_len, -1),
                               dtype=torch.uint8, device=self.device)
+        # one output buffer for the largest batch; a step writes its first rows
+        self.out_buf = torch.empty((cfg.max_num_seqs, cfg.num_q_heads, cfg.head_dim),
+                                   dtype=torch.float32, device=self.device)
+        self.staging = _Staging(self.device)
+        self._ops: List[tuple] = []   # this step's GPU work, in issue order
 
     # ------------------------------------------------------------ helpers
     def _randn(self, shape) -> torch.Tensor:
@@ -111,19 +165,38 @@ class DecodeLoop:
         return r
 
     def _write(self, k: torch.Tensor, v: torch.Tensor, slots: np.ndarray) -> None:
-        st = torch.from_numpy(slots).to(self.device)
-        pa_reshape_and_cache(k, v, self.k_cache, self.v_cache, st)
+        """Queue a cache write (issued in order by _launch)."""
+        self._ops.append(("write", k, v, slots))
         if self.record:
             self.log.append(("write", k, v, slots.copy()))
 
     def _swap(self, pairs: np.ndarray, out: bool) -> None:
-        pt = torch.from_numpy(pairs).to(self.device)
-        if out:
-            pa_swap_blocks(self.k_host, self.v_host, self.k_cache, self.v_cache, pt)
-        else:
-            pa_swap_blocks(self.k_cache, self.v_cache, self.k_host, self.v_host, pt)
+        """Queue a swap of whole blocks (issued in order by _launch)."""
+        self._ops.append(("swap_out" if out else "swap_in", pairs))
         if self.record:
             self.log.append(("swap_out" if out else "swap_in", pairs.copy()))
+
+    def _launch(self, decode: Optional[tuple]) -> None:
+        """Send every host array of this step in one staged copy, then issue
+        the step's swaps and cache writes in the order they were queued, and
+        the decode last."""
+        arrays = [op[-1] for op in self._ops]
+        if decode is not None:
+            arrays += [decode[0], decode[1]]
+        dev = self.staging.upload(arrays)
+        for op, d in zip(self._ops, dev):
+            if op[0] == "write":
+                pa_reshape_and_cache(op[1], op[2], self.k_cache, self.v_cache, d)
+            elif op[0] == "swap_out":
+                pa_swap_blocks(self.k_host, self.v_host, self.k_cache, self.v_cache, d)
+            else:
+                pa_swap_blocks(self.k_cache, self.v_cache, self.k_host, self.v_host, d)
+        self._ops = []
+        if decode is not None:
+            tables, lens, q, out = decode
+            bt, cl = dev[-2], dev[-1]
+            pa_decode(out, q, self.k_cache, self.v_cache, bt, cl, int(lens.max()),
+                      self.sm_scale, workspace=self.ws)
 
     def _preempt(self, keep: Optional[Request]) -> bool:
         """Swap out the most recently admitted running request other than
@@ -198,17 +271,16 @@ class DecodeLoop:
             assert len(cow) == 0  # the loop never forks, so nothing is shared
         stats = {"step": self.step_no, "running": n, "waiting": len(self.waiting),
                  "swapped": len(self.swapped)}
+        decode = None
         if n:
             tables, lens = self.pool.block_tables(ids, self.width)
             kv_shape = (n, c.num_kv_heads, c.head_dim)
             self._write(self._randn(kv_shape), self._randn(kv_shape), slots)
             q = self._randn((n, c.num_q_heads, c.head_dim))
-            out = torch.empty((n, c.num_q_heads, c.head_dim), dtype=torch.float32,
-                              device=self.device)
-            bt = torch.from_numpy(tables).to(self.device)
-            cl = torch.from_numpy(lens).to(self.device)
-            pa_decode(out, q, self.k_cache, self.v_cache, bt, cl, int(lens.max()),
-                      self.sm_scale, workspace=self.ws)
+            out = self.out_buf[:n]
+            decode = (tables, lens, q, out)
+        self._launch(decode)
+        if n:
             for r in batch:
                 r.generated += 1
             held = int(((lens.astype(np.int64) + BS - 1) // BS).sum())
