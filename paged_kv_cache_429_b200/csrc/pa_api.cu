@@ -13,6 +13,7 @@
 #include "pa.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "decode_tc.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -123,6 +124,24 @@ pa_status launch_decode(const void *k_cache, const void *v_cache, int rows,
   if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
   dim3 grid(grid_x, p.num_kv_heads, num_seqs);
   kern<<<grid, pa::kDecodeThreads, smem, stream>>>(tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// The fp8 decode on the 5th-generation tensor core (decode_tc.cuh): head_dim
+// 128, single-pass, one CTA per (sequence, KV head).
+template <int GMAX, bool APPEND>
+pa_status launch_decode_tc(const void *k_cache, const void *v_cache, int rows,
+                           const DecodeParams &p, int num_seqs, cudaStream_t stream, int dev) {
+  CUtensorMap tk, tv;
+  if (!make_cache_tmap<128, true>(&tk, k_cache, rows) ||
+      !make_cache_tmap<128, true>(&tv, v_cache, rows))
+    return PA_ERR_CUDA;
+  auto kern = pa::paged_decode_tc_kernel<GMAX, APPEND>;
+  static std::atomic<uint64_t> attr_done{0};
+  const size_t smem = pa::TdPlan<GMAX>::kSmemBytes;
+  if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
+  dim3 grid(1, p.num_kv_heads, num_seqs);
+  kern<<<grid, pa::kTdThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -331,6 +350,13 @@ static pa_status decode_common(float *out, const void *q, const void *k_cache,
   const bool chunked = psize > 0;
   const int rows = static_cast<int>(rows64);
   pa_status rc;
+  if (kv_dtype == PA_KV_FP8_E4M3 && head_dim == 128 && !chunked && group <= 8) {
+    if (new_k)
+      return group <= 4 ? launch_decode_tc<4, true>(k_cache, v_cache, rows, p, num_seqs, st, dev)
+                        : launch_decode_tc<8, true>(k_cache, v_cache, rows, p, num_seqs, st, dev);
+    return group <= 4 ? launch_decode_tc<4, false>(k_cache, v_cache, rows, p, num_seqs, st, dev)
+                      : launch_decode_tc<8, false>(k_cache, v_cache, rows, p, num_seqs, st, dev);
+  }
   if (kv_dtype == PA_KV_BF16)
     rc = head_dim == 128
              ? dispatch_nt<128, false>(nt, chunked, k_cache, v_cache, rows, p, num_seqs, grid_x, st, dev)

@@ -264,6 +264,50 @@ __device__ __forceinline__ void tc_st_32x32b_x16(uint32_t taddr, const uint32_t 
         "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tc_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tc_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                 "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// N consecutive 32-bit columns of this thread's lane, N a multiple of 8
+// (composed of the x32 / x16 / x8 shapes). Wait with tc_wait_ld before use.
+template <int N>
+__device__ __forceinline__ void tc_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "columns in multiples of 8");
+  if constexpr (N >= 32) {
+    tc_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    if constexpr (N > 32) tc_ld_cols<N - 32>(taddr + 32, *reinterpret_cast<uint32_t(*)[N - 32]>(&r[32]));
+  } else if constexpr (N >= 16) {
+    tc_ld_32x32b_x16(taddr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+    if constexpr (N > 16) tc_ld_cols<N - 16>(taddr + 16, *reinterpret_cast<uint32_t(*)[N - 16]>(&r[16]));
+  } else {
+    tc_ld_32x32b_x8(taddr, *reinterpret_cast<uint32_t(*)[8]>(&r[0]));
+  }
+}
+template <int N>
+__device__ __forceinline__ void tc_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N % 8 == 0, "columns in multiples of 8");
+  tc_st_32x32b_x8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(&r[0]));
+  if constexpr (N > 8) tc_st_cols<N - 8>(taddr + 8, *reinterpret_cast<const uint32_t(*)[N - 8]>(&r[8]));
+}
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -280,6 +324,27 @@ __device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr, uint32_t lbo_b
          (static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
          (2ull << 61);
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::f8f6f4 (operand types from the
+// instruction descriptor; fp32 accumulate), issued by one thread.
+__device__ __forceinline__ void tc_mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4 with E4M3 A and E4M3 (b_e5m2 false)
+// or E5M2 B, fp32 D, M x N tile; each operand K-contiguous unless its
+// mn_major flag is set (an option the 8-bit float formats have).
+__host__ __device__ constexpr uint32_t tc_idesc_f8(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                   bool b_e5m2) {
+  return (1u << 4) | ((b_e5m2 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D, M x N tile;
@@ -307,6 +372,46 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t &lo, uint
       "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(x));
+}
+
+// Two floats -> two E4M3 codes (lo in byte 0, hi in byte 1): round to
+// nearest even, finite values beyond 448 saturated.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t y;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+// Two E4M3 codes (byte 0, byte 1 of x) -> their values as floats (exact).
+__device__ __forceinline__ void e4m3x2_to_f32x2(uint32_t x, float &lo, float &hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}"
+      : "=r"(h2)
+      : "r"(x));
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
+}
+
+// Two floats -> two E5M2 codes (lo in byte 0, hi in byte 1): round to
+// nearest even, finite values beyond 57344 saturated.
+__device__ __forceinline__ uint32_t f32x2_to_e5m2x2(float lo, float hi) {
+  uint16_t y;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+// Two E5M2 codes (byte 0, byte 1 of x) -> their values as floats (exact).
+__device__ __forceinline__ void e5m2x2_to_f32x2(uint32_t x, float &lo, float &hi) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e5m2x2 %0, a;\n\t}"
+      : "=r"(h2)
+      : "r"(x));
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h2));
 }
 
 // Pack two floats into a 16-bit pair (element 0 in the low half), RNE.
