@@ -18,19 +18,21 @@
 //     q_lo = E4M3(2^e q - q_hi), with 2^e per head putting max |q| in
 //     [128, 256): two 4-bit terms hold q's 8 bits exactly (down to the E4M3
 //     subnormal step, 2^-9 of 2^e, where small entries lose a few ulps);
-//   * P (fp32, <= 2^3 by the lazy maximum below) x 2^12 = p1 + .. + p4,
-//     each the E5M2 rounding of what the earlier terms left: ~12
-//     significant bits, and the sum of p over tokens is taken from the same
-//     terms. E5M2, not E4M3: its range keeps the terms of small
-//     probabilities normal (E4M3's subnormal step would cost each token up
-//     to 2^-10 of 2^-6 absolute, which adds up over thousands of tokens).
+//   * P (fp32, <= 2^3 by the lazy maximum below) x 2^12 = p1 + p2 + p3,
+//     each the leading 3 significant bits (one E5M2 value, split off by
+//     Veltkamp's method) of what the earlier terms left: ~9 significant
+//     bits, and the sum of p over tokens is taken from the same terms.
+//     E5M2, not E4M3: its range keeps the terms of small probabilities
+//     normal (E4M3's subnormal step would cost each token up to 2^-10 of
+//     2^-6 absolute, which adds up over thousands of tokens).
 // Per chunk of 128 tokens (8 blocks) and KV head h with group g:
 //   S^T[128 tok][2G]  = K[128 tok][D] . Qs^T             (M 128, N 2G)
 //   softmax over tokens per head (score = column hi + column lo)
-//   O^T[D][4G]       += V^T[D][128 tok] . Ps[128 tok][4G] (M 128 = D, N 4G)
+//   O^T[D][3G]       += V^T[D][128 tok] . Ps[128 tok][3G] (M 128 = D, N 3G
+//                                                           rounded to 8)
 // (G = 4 or 8, the group rounded up; a term's columns start at term * G)
 // with V^T read MN-major from the same [token][dim] tile the TMA wrote, and
-// out = v_scale (sum of O's four term columns) / l at the end.
+// out = v_scale (sum of O's three term columns) / l at the end.
 //
 // Roles (192 threads): warps 0-3 — softmax, one thread per token of the
 // chunk (its tensor-memory lane), and at the end one thread per output
@@ -57,32 +59,36 @@ namespace pa {
 
 constexpr int kTdChunk = 128;               // tokens per chunk: the S MMA's M
 constexpr int kTdBlocks = kTdChunk / kBS;   // blocks per chunk
-constexpr int kTdStages = 3;                // stages of the K ring and of the V ring
+constexpr int kTdKStages = 3;               // K ring stages (freed once S is computed)
+constexpr int kTdVStages = 3;               // V ring stages (freed once PV is computed)
 constexpr int kTdProducerWarp = 4;
 constexpr int kTdMmaWarp = 5;
 constexpr int kTdThreads = 6 * 32;
 constexpr float kTdLazyLog2 = 3.f;          // raise the max only past 2^3
 constexpr float kTdPScale = 4096.f;         // P (<= 8) x 2^12 <= 2^15 < 57344
-constexpr int kTdPTerms = 4;                // E5M2 terms of P
+constexpr int kTdPTerms = 3;                // E5M2 terms of P
+constexpr int kTdOrderMaxSeqs = 256;        // longest-first order up to this batch size
 
 template <int GMAX>
 struct TdPlan {
   // columns (term, head) at term * GMAX + head; heads >= g hold zeros
   static constexpr int kNQ = (2 * GMAX + 7) / 8 * 8;  // score columns: 2 terms
-  static constexpr int kNP = (kTdPTerms * GMAX + 7) / 8 * 8;  // PV columns: 4 terms
+  static constexpr int kNP = (kTdPTerms * GMAX + 7) / 8 * 8;  // PV columns: 3 terms
   static constexpr int kTile = kTdChunk * 128;        // a chunk's K (or V): 128 rows x 128 B
   static constexpr int kKOff = 0;
-  static constexpr int kVOff = kTdStages * kTile;
-  static constexpr int kQOff = 2 * kTdStages * kTile;
+  static constexpr int kVOff = kTdKStages * kTile;
+  static constexpr int kQOff = (kTdKStages + kTdVStages) * kTile;
   static constexpr int kQBytes = (kNQ + 7) / 8 * 1024;  // 8-row, 1 KB swizzle atoms
   static constexpr int kPOff = kQOff + kQBytes;
   static constexpr int kPBytes = (kNP + 7) / 8 * 1024;
   // per-warp partial maxima of two chunks, sums and q maxima
   static constexpr int kRedOff = kPOff + 2 * kPBytes;
   static constexpr int kRedFloats = 2 * 4 * GMAX + 4 * GMAX + 4 * GMAX;
-  static constexpr int kBarOff = kRedOff + kRedFloats * 4;
-  // k_full[3] k_empty[3] v_full[3] v_empty[3] q_ready s_full[2] p_full[2] p_free[2] drain
-  static constexpr int kNumBars = 4 * kTdStages + 1 + 6 + 1;
+  // context lengths of the batch, for the longest-first order
+  static constexpr int kLensOff = kRedOff + kRedFloats * 4;
+  static constexpr int kBarOff = kLensOff + kTdOrderMaxSeqs * 4 + 8;
+  // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] q_ready s_full[2] p_full[2] p_free[2] drain
+  static constexpr int kNumBars = 2 * kTdKStages + 2 * kTdVStages + 1 + 6 + 1;
   static constexpr int kSmemBytes = 1024 + kBarOff + 8 * kNumBars + 16;
   static constexpr int kSCol = 0;                     // S buffer b at kSCol + b * kNQ
   static constexpr int kOCol = 2 * kNQ;
@@ -114,9 +120,8 @@ __device__ __forceinline__ void td_max_heads(float (&v)[GMAX], int g, float *red
 #pragma unroll
   for (int hh = 0; hh < GMAX; ++hh) {
     if (hh >= g) break;
-    float x = v[hh];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    float x;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(x) : "f"(v[hh]));
     if (lane == 0) red[warp * GMAX + hh] = x;
   }
   asm volatile("bar.sync 3, 128;" ::: "memory");
@@ -134,7 +139,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   using TP = TdPlan<GMAX>;
   constexpr int NQ = TP::kNQ;
   constexpr int NP = TP::kNP;
-  constexpr int NS = kTdStages;
+  constexpr int NK = kTdKStages;
+  constexpr int NV = kTdVStages;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -146,10 +152,10 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   const uint32_t sp = base + TP::kPOff;   // split P buffer b at sp + b * kPBytes
   float *red = reinterpret_cast<float *>(base_ptr + TP::kRedOff);
   const uint32_t bar_k_full = base + TP::kBarOff;
-  const uint32_t bar_k_empty = bar_k_full + 8 * NS;
-  const uint32_t bar_v_full = bar_k_empty + 8 * NS;
-  const uint32_t bar_v_empty = bar_v_full + 8 * NS;
-  const uint32_t bar_q = bar_v_empty + 8 * NS;
+  const uint32_t bar_k_empty = bar_k_full + 8 * NK;
+  const uint32_t bar_v_full = bar_k_empty + 8 * NK;
+  const uint32_t bar_v_empty = bar_v_full + 8 * NV;
+  const uint32_t bar_q = bar_v_empty + 8 * NV;
   const uint32_t bar_s_full = bar_q + 8;      // [2]
   const uint32_t bar_p_full = bar_s_full + 16;  // [2]
   const uint32_t bar_p_free = bar_p_full + 16;  // [2]
@@ -158,7 +164,31 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int h = blockIdx.y;
-  const int s = blockIdx.z;
+  // Longest first: CTA z takes the sequence of rank z by context length
+  // (ties by index), so the last CTAs to start are the shortest and the
+  // grid's tail, when too few CTAs remain to keep DRAM busy, is short. The
+  // rank costs a pass over the batch's lengths per CTA (S^2 / 192 compares),
+  // so batches of more than kTdOrderMaxSeqs sequences keep the grid order.
+  int s = blockIdx.z;
+  if (gridDim.z > 1 && gridDim.z <= kTdOrderMaxSeqs) {
+    int *lens = reinterpret_cast<int *>(base_ptr + TP::kLensOff);
+    int *pick = lens + kTdOrderMaxSeqs;
+    const int cap = min(p.max_context_len, p.max_blocks_per_seq * kBS);
+    const int S = static_cast<int>(gridDim.z);
+    for (int i = threadIdx.x; i < S; i += kTdThreads) lens[i] = min(max(p.context_lens[i], 0), cap);
+    __syncthreads();
+    for (int i = threadIdx.x; i < S; i += kTdThreads) {
+      const int li = lens[i];
+      int rank = 0;
+      for (int j = 0; j < S; ++j) {
+        const int lj = lens[j];
+        rank += (lj > li) || (lj == li && j < i);
+      }
+      if (rank == static_cast<int>(blockIdx.z)) *pick = i;
+    }
+    __syncthreads();
+    s = *pick;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = p.group;
@@ -170,9 +200,11 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   if (bad_len && threadIdx.x == 0) raise_error(kErrContextClamp);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NK; ++i) {
       mbar_init(bar_k_full + 8u * i, 1);
       mbar_init(bar_k_empty + 8u * i, 1);
+    }
+    for (int i = 0; i < NV; ++i) {
       mbar_init(bar_v_full + 8u * i, 1);
       mbar_init(bar_v_empty + 8u * i, 1);
     }
@@ -224,8 +256,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         }
       }
       if (lane == 0) {
-        const int st = c % NS;
-        if (c >= NS) ok = tc_wait(bar_k_empty + 8u * st, ((c / NS) - 1) & 1, s_abort);
+        int st = c % NK;
+        if (c >= NK) ok = tc_wait(bar_k_empty + 8u * st, ((c / NK) - 1) & 1, s_abort);
         if (ok) {
           const uint32_t full = bar_k_full + 8u * st;
           mbar_arrive_expect_tx(full, TP::kTile);
@@ -234,7 +266,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
             tma_load_2d(sk + st * TP::kTile + b * 2048, &tmap_k, full, 0, y[b]);
           issued_k = c + 1;
         }
-        if (ok && c >= NS) ok = tc_wait(bar_v_empty + 8u * st, ((c / NS) - 1) & 1, s_abort);
+        st = c % NV;
+        if (ok && c >= NV) ok = tc_wait(bar_v_empty + 8u * st, ((c / NV) - 1) & 1, s_abort);
         if (ok) {
           const uint32_t full = bar_v_full + 8u * st;
           mbar_arrive_expect_tx(full, TP::kTile);
@@ -249,10 +282,10 @@ __global__ void __launch_bounds__(kTdThreads, 2)
     if (lane == 0) {
       if (bad_id) raise_error(kErrBlockRange);
       // no bulk copy may still be landing when the CTA exits
-      for (int c = max(0, issued_k - NS); c < issued_k; ++c)
-        mbar_wait_bounded(bar_k_full + 8u * (c % NS), (c / NS) & 1, kWaitLimitNs);
-      for (int c = max(0, issued_v - NS); c < issued_v; ++c)
-        mbar_wait_bounded(bar_v_full + 8u * (c % NS), (c / NS) & 1, kWaitLimitNs);
+      for (int c = max(0, issued_k - NK); c < issued_k; ++c)
+        mbar_wait_bounded(bar_k_full + 8u * (c % NK), (c / NK) & 1, kWaitLimitNs);
+      for (int c = max(0, issued_v - NV); c < issued_v; ++c)
+        mbar_wait_bounded(bar_v_full + 8u * (c % NV), (c / NV) & 1, kWaitLimitNs);
     }
   } else if (warp == kTdMmaWarp) {
     // ----------------------------------------------------------------- MMA
@@ -287,8 +320,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
     if (nc > 0) {
       bool ok = __all_sync(0xffffffffu, tc_wait(bar_q, 0, s_abort));
       auto issue_s = [&](int c) {
-        const int st = c % NS;
-        ok = __all_sync(0xffffffffu, tc_wait(bar_k_full + 8u * st, (c / NS) & 1, s_abort));
+        const int st = c % NK;
+        ok = __all_sync(0xffffffffu, tc_wait(bar_k_full + 8u * st, (c / NK) & 1, s_abort));
         if (!ok) return;
         const uint32_t kst = sk + st * TP::kTile;
         if (APPEND && c == new_chunk) {
@@ -313,8 +346,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
       for (int c = 0; c < nc && ok; ++c) {
         ok = __all_sync(0xffffffffu, tc_wait(bar_p_full + 8u * (c & 1), (c >> 1) & 1, s_abort));
         if (!ok) break;
-        const int st = c % NS;
-        ok = __all_sync(0xffffffffu, tc_wait(bar_v_full + 8u * st, (c / NS) & 1, s_abort));
+        const int st = c % NV;
+        ok = __all_sync(0xffffffffu, tc_wait(bar_v_full + 8u * st, (c / NV) & 1, s_abort));
         if (!ok) break;
         const uint32_t vst = sv + st * TP::kTile;
         if (APPEND && c == new_chunk) {
@@ -402,6 +435,10 @@ __global__ void __launch_bounds__(kTdThreads, 2)
       mbar_arrive(bar_q);
     }
 
+    // column t of a swizzled 128-byte row, for each row index in its atom
+    int col_off[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) col_off[x] = ((((t >> 4) ^ x) & 7) << 4) + (t & 15);
     // the block holding the context's last, partly filled slots: its V rows
     // past the end may hold NaN codes and are zeroed before PV reads them
     const int tail = L % kBS;
@@ -455,8 +492,10 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         tc_st_cols<NP>(trow + TP::kOCol, o);
         tc_wait_st();
       }
-      // P x 2^12 as four E5M2 terms per head
-      uint32_t pbt[kTdPTerms][GMAX];
+      // P x 2^12 as three E5M2 terms per head: each term is the leading 3
+      // significant bits of what is left (Veltkamp's split with the factor
+      // 2^21 + 1), so it converts to E5M2 exactly, two heads per convert
+      float term[kTdPTerms][GMAX];
 #pragma unroll
       for (int hh = 0; hh < GMAX; ++hh) {
         lpart[hh] *= alpha[hh];
@@ -464,12 +503,11 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         float x = pv * kTdPScale, sum = 0.f;
 #pragma unroll
         for (int k = 0; k < kTdPTerms; ++k) {
-          const uint32_t code = f32x2_to_e5m2x2(x, 0.f) & 0xFFu;
-          float v, unused;
-          e5m2x2_to_f32x2(code, v, unused);
-          pbt[k][hh] = code;
-          sum += v;
-          x -= v;
+          const float gmm = __fmul_rn(x, 2097153.f);
+          const float hi = __fsub_rn(gmm, __fsub_rn(gmm, x));
+          term[k][hh] = hi;
+          sum = __fadd_rn(sum, hi);
+          x = __fsub_rn(x, hi);
         }
         lpart[hh] += sum;
       }
@@ -478,8 +516,8 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         ok = __all_sync(0xffffffffu,
                         tc_wait(bar_p_free + 8u * (c & 1), ((c - 2) >> 1) & 1, s_abort));
       if (ok && c == zero_chunk) {
-        const int st = c % NS;
-        ok = __all_sync(0xffffffffu, tc_wait(bar_v_full + 8u * st, (c / NS) & 1, s_abort));
+        const int st = c % NV;
+        ok = __all_sync(0xffffffffu, tc_wait(bar_v_full + 8u * st, (c / NV) & 1, s_abort));
         if (ok) {
           // rows tail..15 of the last block, 8 chunks of 16 bytes each
           const uint32_t vb = sv + st * TP::kTile + (((L - 1) / kBS) % kTdBlocks) * 2048;
@@ -492,8 +530,13 @@ __global__ void __launch_bounds__(kTdThreads, 2)
 #pragma unroll
       for (int k = 0; k < kTdPTerms; ++k)
 #pragma unroll
-        for (int hh = 0; hh < GMAX; ++hh)
-          if (hh < g) pbuf[sw128_offset(k * GMAX + hh, t)] = static_cast<uint8_t>(pbt[k][hh]);
+        for (int hh = 0; hh < GMAX; hh += 2) {
+          const uint32_t codes = f32x2_to_e5m2x2(term[k][hh], term[k][hh + 1]);
+          const int r = k * GMAX + hh;
+          pbuf[(r >> 3) * 1024 + (r & 7) * 128 + col_off[r & 7]] = static_cast<uint8_t>(codes);
+          pbuf[((r + 1) >> 3) * 1024 + ((r + 1) & 7) * 128 + col_off[(r + 1) & 7]] =
+              static_cast<uint8_t>(codes >> 8);
+        }
       fence_proxy_async_smem();
       tc_fence_before_sync();
       mbar_arrive(bar_p_full + 8u * (c & 1));
@@ -526,7 +569,7 @@ __global__ void __launch_bounds__(kTdThreads, 2)
           const float l = (red_sum[hh] + red_sum[GMAX + hh]) +
                           (red_sum[2 * GMAX + hh] + red_sum[3 * GMAX + hh]);
           const float acc = (__uint_as_float(o[hh]) + __uint_as_float(o[GMAX + hh])) +
-                            (__uint_as_float(o[2 * GMAX + hh]) + __uint_as_float(o[3 * GMAX + hh]));
+                            __uint_as_float(o[2 * GMAX + hh]);
           out[hh * 128] = l > 0.f ? acc * (p.out_scale / l) : 0.f;
         }
       }
