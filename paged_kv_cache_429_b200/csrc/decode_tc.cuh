@@ -34,11 +34,12 @@
 // with V^T read MN-major from the same [token][dim] tile the TMA wrote, and
 // out = v_scale (sum of O's three term columns) / l at the end.
 //
-// Roles (192 threads): warps 0-3 — softmax, one thread per token of the
+// Roles (224 threads): warps 0-3 — softmax, one thread per token of the
 // chunk (its tensor-memory lane), and at the end one thread per output
-// dimension (the lane of O^T); warp 4 — producer (TMA loads of the chunk's
-// 8 K tiles and 8 V tiles into two 3-stage rings, through the table);
-// warp 5 — tensor-memory allocation and the MMA issue (one thread). The
+// dimension (the lane of O^T); warps 4 and 6 — producers (TMA loads of the
+// chunk's 8 K tiles, and of its 8 V tiles, into a K ring and a V ring,
+// through the table); warp 5 — tensor-memory allocation and the MMA issue
+// (one thread). The
 // score buffers are double-buffered, so S for chunk c+1 is computed while
 // the softmax works on chunk c; P has two buffers for the same reason.
 // The running maximum is raised only when a chunk's maximum exceeds it by
@@ -61,9 +62,10 @@ constexpr int kTdChunk = 128;               // tokens per chunk: the S MMA's M
 constexpr int kTdBlocks = kTdChunk / kBS;   // blocks per chunk
 constexpr int kTdKStages = 3;               // K ring stages (freed once S is computed)
 constexpr int kTdVStages = 3;               // V ring stages (freed once PV is computed)
-constexpr int kTdProducerWarp = 4;
+constexpr int kTdKWarp = 4;                 // K producer
 constexpr int kTdMmaWarp = 5;
-constexpr int kTdThreads = 6 * 32;
+constexpr int kTdVWarp = 6;                 // V producer
+constexpr int kTdThreads = 7 * 32;
 constexpr float kTdLazyLog2 = 3.f;          // raise the max only past 2^3
 constexpr float kTdPScale = 4096.f;         // P (<= 8) x 2^12 <= 2^15 < 57344
 constexpr int kTdPTerms = 3;                // E5M2 terms of P
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   // Longest first: CTA z takes the sequence of rank z by context length
   // (ties by index), so the last CTAs to start are the shortest and the
   // grid's tail, when too few CTAs remain to keep DRAM busy, is short. The
-  // rank costs a pass over the batch's lengths per CTA (S^2 / 192 compares),
+  // rank costs a pass over the batch's lengths per CTA (S^2 / 224 compares),
   // so batches of more than kTdOrderMaxSeqs sequences keep the grid order.
   int s = blockIdx.z;
   if (gridDim.z > 1 && gridDim.z <= kTdOrderMaxSeqs) {
@@ -227,16 +229,22 @@ __global__ void __launch_bounds__(kTdThreads, 2)
   tc_fence_after_sync();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == kTdProducerWarp) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
-    }
+  if (warp == kTdKWarp || warp == kTdVWarp) {
+    // --------------------------------------------------------- producers
+    // one warp streams the K tiles, the other the V tiles: the K ring is
+    // freed as soon as S is computed, so its loads never queue behind a V
+    // stage still waiting for its PV
+    const bool is_k = warp == kTdKWarp;
+    const CUtensorMap *tmap = is_k ? &tmap_k : &tmap_v;
+    const int nst = is_k ? NK : NV;
+    const uint32_t ring = is_k ? sk : sv;
+    const uint32_t bar_full = is_k ? bar_k_full : bar_v_full;
+    const uint32_t bar_empty = is_k ? bar_k_empty : bar_v_empty;
+    if (lane == 0) prefetch_tmap(tmap);
     const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
     const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
     bool ok = true, bad_id = false;
-    int issued_k = 0, issued_v = 0;
+    int issued = 0;
     int mine = -1;
     for (int c = 0; c < nc && ok; ++c) {
       if ((c & 3) == 0) {  // 32 table entries: four chunks
@@ -256,36 +264,24 @@ __global__ void __launch_bounds__(kTdThreads, 2)
         }
       }
       if (lane == 0) {
-        int st = c % NK;
-        if (c >= NK) ok = tc_wait(bar_k_empty + 8u * st, ((c / NK) - 1) & 1, s_abort);
+        const int st = c % nst;
+        if (c >= nst) ok = tc_wait(bar_empty + 8u * st, ((c / nst) - 1) & 1, s_abort);
         if (ok) {
-          const uint32_t full = bar_k_full + 8u * st;
+          const uint32_t full = bar_full + 8u * st;
           mbar_arrive_expect_tx(full, TP::kTile);
 #pragma unroll
           for (int b = 0; b < kTdBlocks; ++b)
-            tma_load_2d(sk + st * TP::kTile + b * 2048, &tmap_k, full, 0, y[b]);
-          issued_k = c + 1;
-        }
-        st = c % NV;
-        if (ok && c >= NV) ok = tc_wait(bar_v_empty + 8u * st, ((c / NV) - 1) & 1, s_abort);
-        if (ok) {
-          const uint32_t full = bar_v_full + 8u * st;
-          mbar_arrive_expect_tx(full, TP::kTile);
-#pragma unroll
-          for (int b = 0; b < kTdBlocks; ++b)
-            tma_load_2d(sv + st * TP::kTile + b * 2048, &tmap_v, full, 0, y[b]);
-          issued_v = c + 1;
+            tma_load_2d(ring + st * TP::kTile + b * 2048, tmap, full, 0, y[b]);
+          issued = c + 1;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (lane == 0) {
-      if (bad_id) raise_error(kErrBlockRange);
+      if (bad_id && is_k) raise_error(kErrBlockRange);
       // no bulk copy may still be landing when the CTA exits
-      for (int c = max(0, issued_k - NK); c < issued_k; ++c)
-        mbar_wait_bounded(bar_k_full + 8u * (c % NK), (c / NK) & 1, kWaitLimitNs);
-      for (int c = max(0, issued_v - NV); c < issued_v; ++c)
-        mbar_wait_bounded(bar_v_full + 8u * (c % NV), (c / NV) & 1, kWaitLimitNs);
+      for (int c = max(0, issued - nst); c < issued; ++c)
+        mbar_wait_bounded(bar_full + 8u * (c % nst), (c / nst) & 1, kWaitLimitNs);
     }
   } else if (warp == kTdMmaWarp) {
     // ----------------------------------------------------------------- MMA
