@@ -603,6 +603,14 @@ def run_loop(args):
     live = [st for st in stats if st["running"]]
     tokens = sum(st["running"] for st in live)
     mean = lambda k: sum(st[k] for st in live) / max(len(live), 1)
+    # the decode's algorithmic bytes per step (K and V of every context
+    # token, q, out, table entries, lengths) and its time at the copy peak
+    eb = 2
+    dec_bytes = [st["tokens"] * cfg.num_kv_heads * cfg.head_dim * eb * 2
+                 + st["running"] * cfg.num_q_heads * cfg.head_dim * 6
+                 + st["blocks_held"] * 4 + 4 * st["running"] for st in live]
+    peak, peak_src = measured_peak()
+    bound_ms = 1e3 * (sum(dec_bytes) / max(len(stats), 1)) / (peak * 1e9)
     return {
         "op": "loop", "metric": "continuous-batching decode loop: decode tokens/s "
         "(one attention layer, host scheduling included)",
@@ -617,6 +625,10 @@ def run_loop(args):
         "kv_utilisation_reserved_max_len": round(mean("reserved_util"), 4),
         "min_kv_utilisation_paged": round(min(st["paged_util"] for st in live), 4),
         "preemptions": loop.preemptions, "finished": loop.finished,
+        "decode_gb_per_step": round(sum(dec_bytes) / max(len(stats), 1) / 1e9, 4),
+        "decode_at_peak_ms_per_step": round(bound_ms, 4),
+        "step_over_decode_at_peak": round((1e3 * secs / args.steps) / bound_ms, 3) if bound_ms else None,
+        "peak_gbs": peak, "peak_source": peak_src,
     }
 
 

@@ -36,7 +36,10 @@
 //     1-3 hand theirs to warp 0 through shared memory, and warp 0 writes
 //     either the normalised output (single-pass) or the partition's
 //     unnormalised output with its max and sum (split; a second kernel
-//     combines the partitions).
+//     combines the partitions). The split path's partial outputs are
+//     written with an L2 evict-last policy and the combining kernel drops
+//     them from L2 after reading them, so they normally never travel to
+//     DRAM and back.
 // With the step's new tokens fused in (pa_decode_append), the CTA holding a
 // sequence's last block first writes the new token's K/V row of its KV head
 // into slot L - 1 (as reshape_and_cache would), then streams as above.
@@ -464,6 +467,7 @@ __device__ __forceinline__ void merge_and_write(WarpState<D, NT> &ws, float *mbu
   combine_record<D, NT>(ws, mbuf + lane * LF);
 
   const int group = p.group;
+  const uint64_t pol = l2_evict_last_policy();
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int n0 = nt * 8 + 2 * qd;
@@ -497,8 +501,13 @@ __device__ __forceinline__ void merge_and_write(WarpState<D, NT> &ws, float *mbu
           d0 = 16 * mt + 2 * gq;
           d1 = d0 + 1;
         }
-        dst[d0] = ws.acc[nt][mt][c] * scale;
-        dst[d1] = ws.acc[nt][mt][2 + c] * scale;
+        if (split) {  // the reduce reads it back soon: keep it in L2
+          st_global_f32_hint(dst + d0, ws.acc[nt][mt][c] * scale, pol);
+          st_global_f32_hint(dst + d1, ws.acc[nt][mt][2 + c] * scale, pol);
+        } else {
+          dst[d0] = ws.acc[nt][mt][c] * scale;
+          dst[d1] = ws.acc[nt][mt][2 + c] * scale;
+        }
       }
     }
   }
@@ -933,6 +942,13 @@ __global__ void __launch_bounds__(kReduceWarps * 32) paged_decode_reduce_kernel(
     }
     out[tid] = a / t;
   }
+  // Every partial output of this (sequence, head) has been read: drop its
+  // lines from L2 without writing them back to DRAM (the workspace holds
+  // nothing a later call reads). Its partial maxima and sums share lines
+  // with other heads' and stay.
+  __syncthreads();
+  const char *ob = reinterpret_cast<const char *>(p.ws_o + row0 * D);
+  for (int i = tid; i < P * (D * 4 / 128); i += kReduceWarps * 32) discard_l2_line(ob + 128 * i);
 }
 
 }  // namespace pa
