@@ -50,6 +50,7 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20
 DECODE_SOURCES = ["paged_kv_cache_429_b200/csrc/decode.cuh",
+                  "paged_kv_cache_429_b200/csrc/decode_tc.cuh",
                   "paged_kv_cache_429_b200/csrc/kv_quant.cuh",
                   "paged_kv_cache_429_b200/csrc/ptx.cuh"]
 

@@ -170,6 +170,22 @@ __device__ __forceinline__ int clamped_len(const int32_t *context_lens, int s,
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
+// Bounded wait shared by the roles of the tensor-core kernels; on time-out flags the error and the
+// CTA-wide abort word. Returns false if the wait failed or the CTA aborted.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      raise_error(kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
 // Named barriers: 1 = the four consumer warps, 2 = consumer warps 0 and 1.
 __device__ __forceinline__ void consumer_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");

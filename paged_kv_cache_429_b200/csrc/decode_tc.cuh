@@ -54,7 +54,6 @@
 #pragma once
 
 #include "decode.cuh"
-#include "prefill.cuh"
 
 namespace pa {
 

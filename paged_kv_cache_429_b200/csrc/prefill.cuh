@@ -97,22 +97,6 @@ struct TcPlan {
   static_assert(kSmemBytes <= 227 * 1024, "shared-memory plan");
 };
 
-// Bounded wait shared by all roles; on time-out flags the error and the
-// CTA-wide abort word. Returns false if the wait failed or the CTA aborted.
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      raise_error(kErrWaitTimeout);
-      return false;
-    }
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
