@@ -93,16 +93,21 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, partition_size: int = None):
     """DRAM bytes per decode launch from the committed ncu summary of this
-    workload, if it was taken on the current decode kernel source."""
+    workload (the entry for this partition size when the summary has one),
+    if it was taken on the current decode kernel source."""
     path = os.path.join(ROOT, "profiles", f"paged_decode_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    m_tr = None
+    if partition_size is not None:
+        m_tr = re.search(r"dram_bytes_per_launch_ps%d:\s*([0-9]+)" % partition_size, text)
+    if m_tr is None:
+        m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
     if not (m_hash and m_tr) or m_hash.group(1) != decode_source_hash():
         return None
     return int(m_tr.group(1))
@@ -371,7 +376,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(w.name),
+                     "traffic": profiled_traffic(w.name, ps),
                      "kernel": "paged_decode_kernel" + (" (new-token write fused)" if fuse else "")
                                + (" + reduce" if split else ""),
                      "algorithmic_bytes_per_launch": kernel_bytes,

@@ -48,6 +48,25 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("missing") is None
 
 
+def test_traffic_per_partition_size(tmp_path, monkeypatch):
+    """A summary with entries per partition size gives each path its own
+    bytes, and the plain entry when the size has none."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "decode_source_hash", lambda: "0123456789abcdef")
+    _profile(tmp_path, "split", "decode_source_sha256_16: 0123456789abcdef\n"
+                                "dram_bytes_per_launch_ps512: 3669506560\n"
+                                "dram_bytes_per_launch_ps-1: 3598697472\n")
+    _profile(tmp_path, "both", "decode_source_sha256_16: 0123456789abcdef\n"
+                               "dram_bytes_per_launch: 100\n"
+                               "dram_bytes_per_launch_ps512: 200\n")
+    assert bench.profiled_traffic("split", 512) == 3669506560
+    assert bench.profiled_traffic("split", -1) == 3598697472
+    assert bench.profiled_traffic("split", 0) is None
+    assert bench.profiled_traffic("both", 512) == 200
+    assert bench.profiled_traffic("both", 0) == 100
+    assert bench.profiled_traffic("both") == 100
+
+
 def _run_main(argv, capsys, monkeypatch, env=None):
     for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
         monkeypatch.delenv(k, raising=False)
