@@ -91,7 +91,7 @@ struct TcPlan {
   // tile s_full[2], p_full[2], pv_done[2]; drain
   static constexpr int kNumBars = 1 + 2 * kTcKStages + 2 * kTcVStages + 6 * kTcQTiles + 1;
   static constexpr int kSmemBytes = 1024 + kBarOff + 8 * kNumBars + 16;
-  static constexpr int kTmemCols = 512;
+  static constexpr int kTmemCols = kTcQTiles > 1 ? 512 : 256;
   static constexpr int kOCol = 2 * kTcQTiles * kTcKeys;    // O_g at kOCol + g * D
   static_assert(kOCol + kTcQTiles * D <= kTmemCols, "tensor-memory plan");
   static_assert(kSmemBytes <= 227 * 1024, "shared-memory plan");
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (bad_len && threadIdx.x == 0 && qt == 0) raise_error(kErrContextClamp);
   const int group = p.group;
   const int ctx0 = L - n;                           // position of chunk token 0
-  const bool has1 = t0 + tpt < n;                   // query tile 1 has tokens
+  const bool has1 = kTcQTiles > 1 && t0 + tpt < n;  // query tile 1 has tokens
   // key tiles each query tile needs (keys up to its last token's position)
   int nt_g[kTcQTiles];
 #pragma unroll
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int tb = t0 + g * tpt;
     nt_g[g] = tb < n ? (ctx0 + min(n, tb + tpt) - 1) / kTcKeys + 1 : 0;
   }
-  const int ntiles = has1 ? nt_g[1] : nt_g[0];      // key tiles the CTA streams
+  const int ntiles = has1 ? nt_g[kTcQTiles - 1] : nt_g[0];  // key tiles the CTA streams
   const int kmax = ctx0 + min(n, t0 + kTcQTiles * tpt) - 1;
   const int nblk = kmax / kBS + 1;
 

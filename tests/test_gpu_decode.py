@@ -137,6 +137,29 @@ def test_edge_lengths_heads_dtypes(D, fp8, hq, hkv):
     check_batch(b, paths=(0, 16, 512, -1))
 
 
+def test_fp8_tensor_core_order_ties_and_large_batches():
+    """The fp8 tensor-core decode ranks sequences by length (longest first)
+    in batches of up to 256 and keeps the grid order beyond: equal lengths
+    (ties broken by index), a batch of exactly 256, and one of 300 short
+    sequences, every output against the oracle."""
+    for S, lens in ((12, [640] * 6 + [129] * 6),
+                    (256, np.random.default_rng(21).integers(1, 400, size=256)),
+                    (300, np.random.default_rng(22).integers(1, 300, size=300))):
+        w = synth.Workload(f"order{S}", S, 8, 2, 128, True, pool_factor=1.3)
+        b = DecodeBatch.build(w, 4, lens=np.asarray(lens))
+        check_batch(b, paths=(0,))
+
+
+def test_fp8_tensor_core_chunk_boundaries():
+    """Lengths on and around the 128-token chunks of the fp8 tensor-core
+    decode, with GQA groups of 1, 4 and 8 (two instances of the kernel)."""
+    lens = np.array([127, 128, 129, 255, 256, 257, 383, 384, 385, 1, 17, 8192])
+    for hq, hkv in ((4, 4), (16, 4), (16, 2)):
+        w = synth.Workload(f"chunks{hq}{hkv}", len(lens), hq, hkv, 128, True, pool_factor=1.2)
+        b = DecodeBatch.build(w, 9, lens=lens)
+        check_batch(b, paths=(0, -1))
+
+
 SPLIT_EDGE_LENS = [1, 2, 15, 16, 17, 511, 512, 513, 1024, 1025, 2047, 2048, 2049, 2560, 3000,
                    3072]
 
