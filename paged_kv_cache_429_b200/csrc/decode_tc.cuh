@@ -293,25 +293,36 @@ __global__ void __launch_bounds__(kTdThreads, 2)
     int new_chunk = -1;       // chunk holding the new token (position L - 1)
     uint32_t new_off = 0;     // its row's offset inside the chunk's tile
     uint2 new_k8 = make_uint2(0u, 0u), new_v8 = new_k8;  // lanes 0-15: 8 E4M3 codes each
+    // The new row's loads are issued here; quantising it (IEEE divisions)
+    // and storing it to the cache wait until the warp would otherwise idle
+    // for the softmax: after the first PV, or before the first scores when
+    // the token falls in the first two chunks.
+    uint4 new_kx = make_uint4(0u, 0u, 0u, 0u), new_vx = new_kx;
+    int new_pid = -1;
     if (APPEND && L > 0 && !bad_len) {
       const int pos = L - 1;
       new_chunk = pos / kTdChunk;
       new_off = ((pos % kTdChunk) / kBS) * 2048 + (pos % kBS) * 128;
-      const int pid = p.block_tables[static_cast<int64_t>(s) * p.max_blocks_per_seq + pos / kBS];
+      new_pid = p.block_tables[static_cast<int64_t>(s) * p.max_blocks_per_seq + pos / kBS];
       if (lane < 16) {
         const int64_t src = (static_cast<int64_t>(s) * p.num_kv_heads + h) * 128 + lane * 8;
-        const uint4 kx = *reinterpret_cast<const uint4 *>(p.new_k + src);
-        const uint4 vx = *reinterpret_cast<const uint4 *>(p.new_v + src);
-        new_k8 = e4m3_chunk(kx, p.k_scale);
-        new_v8 = e4m3_chunk(vx, p.v_scale);
-        // an id outside the pool is left alone (its loads read zeros, flagged)
-        if (pid >= 0 && pid < p.num_blocks)
-          store_kv_chunk<true>(kx, vx, p.k_cache, p.v_cache,
-                               ((static_cast<int64_t>(pid) * p.num_kv_heads + h) * kBS + pos % kBS) *
-                                       128 + lane * 8,
-                               p.k_scale, p.v_scale);
+        new_kx = *reinterpret_cast<const uint4 *>(p.new_k + src);
+        new_vx = *reinterpret_cast<const uint4 *>(p.new_v + src);
       }
     }
+    auto write_new_token = [&]() {
+      if (lane < 16) {
+        new_k8 = e4m3_chunk(new_kx, p.k_scale);
+        new_v8 = e4m3_chunk(new_vx, p.v_scale);
+        // an id outside the pool is left alone (its loads read zeros, flagged)
+        if (new_pid >= 0 && new_pid < p.num_blocks)
+          store_kv_chunk<true>(new_kx, new_vx, p.k_cache, p.v_cache,
+                               ((static_cast<int64_t>(new_pid) * p.num_kv_heads + h) * kBS +
+                                (L - 1) % kBS) * 128 + lane * 8,
+                               p.k_scale, p.v_scale);
+      }
+    };
+    if (APPEND && new_chunk >= 0 && new_chunk < 2) write_new_token();
     if (nc > 0) {
       bool ok = __all_sync(0xffffffffu, tc_wait(bar_q, 0, s_abort));
       auto issue_s = [&](int c) {
@@ -361,6 +372,7 @@ __global__ void __launch_bounds__(kTdThreads, 2)
           tc_commit(bar_v_empty + 8u * st);
         }
         __syncwarp();
+        if (APPEND && c == 0 && new_chunk >= 2) write_new_token();
         if (c + 2 < nc) issue_s(c + 2);
       }
       // every MMA issued here has completed before tensor memory is freed
