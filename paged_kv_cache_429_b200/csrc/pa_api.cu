@@ -448,11 +448,11 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
   p.group = group;
-  p.tokens_per_tile = pa::kTcRows / group;
+  p.tokens_per_tile = pa::kPfRows / group;
   p.num_blocks = num_blocks;
   p.score_scale = sm_scale * 1.4426950408889634f;
   const int rows = static_cast<int>(rows64);
-  const int64_t cta_tokens = static_cast<int64_t>(pa::kTcQTiles) * p.tokens_per_tile;
+  const int64_t cta_tokens = static_cast<int64_t>(pa::kPfQTiles) * p.tokens_per_tile;
   const int64_t tiles = (static_cast<int64_t>(max_query_len) + cta_tokens - 1) / cta_tokens;
   if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
@@ -465,19 +465,19 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
         !make_cache_tmap<128, false>(&tv, v_cache, rows))
       return PA_ERR_CUDA;
     auto kern = pa::paged_prefill_kernel<128>;
-    const size_t smem = pa::TcPlan<128>::kSmemBytes;
+    const size_t smem = pa::PfPlan<128>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
-    kern<<<grid, pa::kTcThreads, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, p);
   } else {
     if (!make_cache_tmap<64, false>(&tk, k_cache, rows) ||
         !make_cache_tmap<64, false>(&tv, v_cache, rows))
       return PA_ERR_CUDA;
     auto kern = pa::paged_prefill_kernel<64>;
-    const size_t smem = pa::TcPlan<64>::kSmemBytes;
+    const size_t smem = pa::PfPlan<64>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
-    kern<<<grid, pa::kTcThreads, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, p);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
