@@ -98,6 +98,25 @@ bool make_q_tmap(CUtensorMap *map, const void *q, int num_tokens, int num_q_head
   return r == CUDA_SUCCESS;
 }
 
+// Prefill output rows: a 3-D view [tokens][query heads][head_dim] of the
+// fp32 output, box (32 columns = 128 bytes, the GQA group's heads, tokens
+// of a tile) with the 128-byte swizzle, the layout the kernel stages O in.
+bool make_out_tmap(CUtensorMap *map, float *out, int num_tokens, int num_q_heads, int head_dim,
+                   int group, int tokens_per_tile) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(num_tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 4,
+                           static_cast<cuuint64_t>(num_q_heads) * head_dim * 4};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tokens_per_tile)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <typename Kern>
 bool ensure_smem_attr(Kern kern, size_t bytes, std::atomic<uint64_t> &done, int dev) {
   const uint64_t bit = 1ull << (dev & 63);
@@ -457,8 +476,9 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
   dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  CUtensorMap tq, tk, tv;
-  if (!make_q_tmap(&tq, q, num_tokens, num_q_heads, head_dim, group, p.tokens_per_tile))
+  CUtensorMap tq, tk, tv, to;
+  if (!make_q_tmap(&tq, q, num_tokens, num_q_heads, head_dim, group, p.tokens_per_tile) ||
+      !make_out_tmap(&to, out, num_tokens, num_q_heads, head_dim, group, p.tokens_per_tile))
     return PA_ERR_CUDA;
   if (head_dim == 128) {
     if (!make_cache_tmap<128, false>(&tk, k_cache, rows) ||
@@ -468,7 +488,7 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
     const size_t smem = pa::PfPlan<128>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
-    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, to, p);
   } else {
     if (!make_cache_tmap<64, false>(&tk, k_cache, rows) ||
         !make_cache_tmap<64, false>(&tv, v_cache, rows))
@@ -477,7 +497,7 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
     const size_t smem = pa::PfPlan<64>::kSmemBytes;
     static std::atomic<uint64_t> attr_done{0};
     if (!ensure_smem_attr(kern, smem, attr_done, dev)) return PA_ERR_CUDA;
-    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, pa::kPfThreads, smem, st>>>(tq, tk, tv, to, p);
   }
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -37,10 +37,13 @@
 //     a running max m and sum l in the exp2 domain. The max used for P is
 //     only raised when a row's tile max exceeds it by more than 2^8 (then
 //     O's row is rescaled in tensor memory; PV_g(j-1) has completed once
-//     S_g(j) has), so P <= 2^8. P is rounded to fp16 (11 significant bits)
-//     and written over the first 64 score columns; l sums the rounded
-//     values, the ones the PV MMA multiplies. At the end each thread scales
-//     its O row by 2^8 / l and stores it.
+//     S_g(j) has), so P <= 2^8. The arguments are formed with f32x2 FMAs,
+//     P is rounded to fp16 (11 significant bits) and written over the first
+//     64 score columns, and l sums P in fp32 (f32x2 adds) before rounding.
+//     At the end each thread scales its O row by 2^8 / l; a tile whose
+//     tokens all belong to the chunk is staged through its own Q buffer in
+//     the 128-byte swizzled layout and written by TMA stores (coalesced,
+//     asynchronous), other tiles row by row.
 //   * warp 15 takes part only in the register split (setmaxnreg): the two
 //     softmax warpgroups run with 192 registers, the others with 64.
 // Shared memory (head_dim 128): Q 64 KB, 2 K and 2 V stages of 32 KB:
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                          const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v,
+                         const __grid_constant__ CUtensorMap tmap_o,
                          const PrefillParams p) {
   using TP = PfPlan<D>;
   constexpr int H = TP::kHalves;
@@ -436,7 +440,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
       for (int c = 0; c < kPfKeys; ++c) z[c] = __uint_as_float(sr[c >> 5][c & 31]);
       const int kb = j * kPfKeys;
-      if (kb + kPfKeys - 1 > klim) {
+      // every row of the warp sees every key of the tile: no mask, and no
+      // row without a visible key (the warp takes this branch as one)
+      const bool open = __all_sync(0xffffffffu, kb + kPfKeys - 1 <= klim);
+      if (!open && kb + kPfKeys - 1 > klim) {
 #pragma unroll
         for (int c = 0; c < kPfKeys; ++c)
           if (kb + c > klim) z[c] = -INFINITY;
@@ -458,21 +465,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
       l *= alpha;
       m_used = m_new;
-      // P (fp16 pairs, the lower key in the low half) over the first 64
-      // score columns
+      // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
+      // over the first 64 score columns; l sums P in fp32 before rounding.
+      // Open tiles form the pairs' arguments with one f32x2 FMA; tiles with
+      // masked keys or dead rows go element by element and zero dead rows.
       const bool live = valid && m_used != -INFINITY;
       const float neg_m = -m_used;
-      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[2][32];
+      uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+      // two halves of 64 keys, each stored (32 columns) as soon as it is
+      // packed: its scores are already in registers, and half the packed
+      // registers are live at a time
 #pragma unroll
-      for (int e = 0; e < kPfKeys / 2; ++e) {
-        const float p0 = live ? ex2_approx(fmaf(z[2 * e], scale, neg_m)) : 0.f;
-        const float p1 = live ? ex2_approx(fmaf(z[2 * e + 1], scale, neg_m)) : 0.f;
-        const uint32_t hp = pack2<true>(p0, p1);
-        float r0, r1;
-        unpack2<true>(hp, r0, r1);
-        rsum[e & 3] += r0 + r1;
-        pk[e >> 5][e & 31] = hp;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[32];
+        if (open) {
+          const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = 64 * hh + 2 * e;
+            const uint64_t x = f2_fma(f2(z[c], z[c + 1]), sc2, nm2);
+            float p0, p1;
+            f2_split(x, p0, p1);
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
+            pk[e] = pack2<true>(p0, p1);
+            lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = 64 * hh + 2 * e;
+            const float p0 = live ? ex2_approx(fmaf(z[c], scale, neg_m)) : 0.f;
+            const float p1 = live ? ex2_approx(fmaf(z[c + 1], scale, neg_m)) : 0.f;
+            pk[e] = pack2<true>(p0, p1);
+            lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+          }
+        }
+        tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
       }
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
         // O_g holds PV_g(j-1): it completed before S_g(j)
@@ -486,9 +515,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_st_32x32b_x32(trow + ocol + cc * 32, o);
         }
       }
-      tc_st_32x32b_x32(trow + scol, pk[0]);
-      tc_st_32x32b_x32(trow + scol + 32, pk[1]);
-      l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+      {
+        float a0, a1, b0, b1;
+        f2_split(lsum[0], a0, a1);
+        f2_split(lsum[1], b0, b1);
+        l += (a0 + b0) + (a1 + b1);
+      }
       tc_wait_st();
       tc_fence_before_sync();
       mbar_arrive(bar_p_full + 8u * g);
@@ -496,21 +528,65 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ epilogue
     if (ok && ntg > 0)
       ok = __all_sync(0xffffffffu, tc_wait(bar_o_done + 8u * g, 0, s_abort));
+    // the warpgroup decides together (the staged path below has barriers
+    // over its 128 threads): every warp that reaches here votes
+    if (ntg > 0) ok = named_bar_and(1 + g, 128, ok);
     if (ok && ntg > 0) {
       tc_fence_after_sync();
       const float inv = l > 0.f ? kPfOutScale / l : 0.f;
-      float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
+      if (t0 + g * tpt + tpt <= n) {
+        // Every token of the tile is in the chunk: stage O through this
+        // tile's Q buffer (all of its score MMAs have completed) as boxes of
+        // 32 fp32 columns x the tile's rows in the 128-byte swizzled layout
+        // (thread r writes row r, its 16-byte chunk c at c ^ (r % 8): no bank
+        // conflicts) and write them with TMA stores, H boxes per round.
+        const uint32_t stage = sq + g * TP::kQBytes;
+        const uint32_t bar_id = 1 + g;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
-        tc_wait_ld();
-        if (valid) {
+        for (int rd = 0; rd < 2; ++rd) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(orow + cc * 32 + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          for (int bx = 0; bx < H; ++bx) {
+            const int cc = rd * H + bx;  // 32-column block
+            uint32_t o[32];
+            tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+            tc_wait_ld();
+            const uint32_t rowp = stage + bx * (kPfRows * 128) + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 v;
+              v.x = __float_as_uint(__uint_as_float(o[4 * c]) * inv);
+              v.y = __float_as_uint(__uint_as_float(o[4 * c + 1]) * inv);
+              v.z = __float_as_uint(__uint_as_float(o[4 * c + 2]) * inv);
+              v.w = __float_as_uint(__uint_as_float(o[4 * c + 3]) * inv);
+              st_shared_v4(rowp + ((c ^ (r & 7)) << 4), v);
+            }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(bar_id, 128);
+          if (r == 0) {
+#pragma unroll
+            for (int bx = 0; bx < H; ++bx)
+              tma_store_3d(&tmap_o, stage + bx * (kPfRows * 128), (rd * H + bx) * 32, h * group,
+                           q0 + t0 + g * tpt);
+            bulk_commit_group();
+            bulk_wait_read_all();
+          }
+          named_bar_sync(bar_id, 128);  // the staging buffer may be rewritten
+        }
+      } else {
+        float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+          tc_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(orow + cc * 32 + e) =
+                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          }
         }
       }
     }

@@ -130,6 +130,27 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap,
       : "memory");
 }
 
+// 3-D tiled bulk tensor store shared -> global (x innermost), tracked in
+// this thread's bulk group. Elements of the box outside the tensor are not
+// written; rows inside it are, so a caller stores only boxes it owns.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until every bulk store this thread committed has read its shared
+// memory source (the global writes may still be in flight).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA, tensor core) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -143,6 +164,23 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 }
 __device__ __forceinline__ void st_shared_v2(uint32_t addr, uint2 v) {
   asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Barrier `id` (1..15) over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// The same barrier, returning the AND of `pred` over its threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t y;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(y)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return y != 0;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
@@ -462,6 +500,32 @@ __device__ __forceinline__ void unpack2(uint32_t x, float &lo, float &hi) {
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
   uint32_t y;
   asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(a), "r"(sel));
+  return y;
+}
+
+// ------------------------------------------------------- packed fp32 pairs
+// Two floats in a 64-bit register pair (element 0 in the low half), for the
+// f32x2 add and fused multiply-add of sm_100 (one instruction per pair).
+
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t y;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(lo), "f"(hi));
+  return y;
+}
+
+__device__ __forceinline__ void f2_split(uint64_t x, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t y;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y) : "l"(a), "l"(b), "l"(c));
+  return y;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t y;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(a), "l"(b));
   return y;
 }
 
