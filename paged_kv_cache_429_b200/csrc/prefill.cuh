@@ -443,76 +443,110 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // every row of the warp sees every key of the tile: no mask, and no
       // row without a visible key (the warp takes this branch as one)
       const bool open = __all_sync(0xffffffffu, kb + kPfKeys - 1 <= klim);
-      if (!open && kb + kPfKeys - 1 > klim) {
-#pragma unroll
-        for (int c = 0; c < kPfKeys; ++c)
-          if (kb + c > klim) z[c] = -INFINITY;
-      }
-      // tile max of the raw scores (scale > 0) as a tree of 3-input maxima
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmax3(z[i], z[i + 8], z[i + 16]);
-#pragma unroll
-      for (int c = 24; c + 16 <= kPfKeys; c += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], z[c + i], z[c + 8 + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[kPfKeys - 8 + i]);
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                             fmaxf(mx[6], mx[7])) * scale;
-      const float m_new = (mt > m_used + kPfRescaleLog2) ? mt : m_used;
-      const bool raise = m_new != m_used;
-      const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
-      l *= alpha;
-      m_used = m_new;
-      // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
-      // over the first 64 score columns; l sums P in fp32 before rounding.
-      // Open tiles form the pairs' arguments with one f32x2 FMA; tiles with
-      // masked keys or dead rows go element by element and zero dead rows.
-      const bool live = valid && m_used != -INFINITY;
-      const float neg_m = -m_used;
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-      // two halves of 64 keys, each stored (32 columns) as soon as it is
-      // packed: its scores are already in registers, and half the packed
-      // registers are live at a time
+      // An open tile after the row's first one is taken speculatively: P
+      // is formed against the max already in use while the tile's largest
+      // argument is tracked beside it, so the exponentials (the special-
+      // function unit) do not wait for a max reduction. Only if some row's
+      // largest argument exceeds 2^8 (the max must be raised) is the tile
+      // redone the plain way, which computes the same P as the speculative
+      // pass wherever the max stays.
+      bool redo = true;
+      if (open && __all_sync(0xffffffffu, m_used != -INFINITY)) {
+        const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_used, -m_used);
+        float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t pk[32];
-        if (open) {
-          const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = 64 * hh + 2 * e;
-            const uint64_t x = f2_fma(f2(z[c], z[c + 1]), sc2, nm2);
-            float p0, p1;
-            f2_split(x, p0, p1);
-            p0 = ex2_approx(p0);
-            p1 = ex2_approx(p1);
-            pk[e] = pack2<true>(p0, p1);
-            lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
-          }
-        } else {
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = 64 * hh + 2 * e;
-            const float p0 = live ? ex2_approx(fmaf(z[c], scale, neg_m)) : 0.f;
-            const float p1 = live ? ex2_approx(fmaf(z[c + 1], scale, neg_m)) : 0.f;
+            float x0, x1;
+            f2_split(f2_fma(f2(z[c], z[c + 1]), sc2, nm2), x0, x1);
+            xm[e & 3] = fmax3(xm[e & 3], x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             pk[e] = pack2<true>(p0, p1);
             lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
           }
+          tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
         }
-        tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
+        redo = __any_sync(0xffffffffu,
+                          fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) > kPfRescaleLog2);
+        if (redo) {
+          tc_wait_st();  // the plain pass rewrites the same columns
+          lsum[0] = lsum[1] = f2(0.f, 0.f);
+        }
       }
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        // O_g holds PV_g(j-1): it completed before S_g(j)
+      if (redo) {
+        if (!open && kb + kPfKeys - 1 > klim) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
-          tc_wait_ld();
+          for (int c = 0; c < kPfKeys; ++c)
+            if (kb + c > klim) z[c] = -INFINITY;
+        }
+        // tile max of the raw scores (scale > 0) as a tree of 3-input maxima
+        float mx[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tc_st_32x32b_x32(trow + ocol + cc * 32, o);
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(z[i], z[i + 8], z[i + 16]);
+#pragma unroll
+        for (int c = 24; c + 16 <= kPfKeys; c += 16)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], z[c + i], z[c + 8 + i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[kPfKeys - 8 + i]);
+        const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                               fmaxf(mx[6], mx[7])) * scale;
+        const float m_new = (mt > m_used + kPfRescaleLog2) ? mt : m_used;
+        const bool raise = m_new != m_used;
+        const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
+        l *= alpha;
+        m_used = m_new;
+        // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
+        // over the first 64 score columns; l sums P in fp32 before
+        // rounding. Open tiles form the pairs' arguments with one f32x2
+        // FMA; tiles with masked keys or dead rows go element by element
+        // and zero dead rows. Each half of 64 keys (32 columns) is stored
+        // as soon as it is packed: its scores are already in registers.
+        const bool live = valid && m_used != -INFINITY;
+        const float neg_m = -m_used;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+          if (open) {
+            const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c = 64 * hh + 2 * e;
+              const uint64_t x = f2_fma(f2(z[c], z[c + 1]), sc2, nm2);
+              float p0, p1;
+              f2_split(x, p0, p1);
+              p0 = ex2_approx(p0);
+              p1 = ex2_approx(p1);
+              pk[e] = pack2<true>(p0, p1);
+              lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int c = 64 * hh + 2 * e;
+              const float p0 = live ? ex2_approx(fmaf(z[c], scale, neg_m)) : 0.f;
+              const float p1 = live ? ex2_approx(fmaf(z[c + 1], scale, neg_m)) : 0.f;
+              pk[e] = pack2<true>(p0, p1);
+              lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+            }
+          }
+          tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
+        }
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          // O_g holds PV_g(j-1): it completed before S_g(j)
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc_st_32x32b_x32(trow + ocol + cc * 32, o);
+          }
         }
       }
       {
