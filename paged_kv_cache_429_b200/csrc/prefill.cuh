@@ -125,10 +125,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return y;
 }
 
-// Eight bf16 (a 16-byte chunk) -> eight fp16 of the values times 2^-8.
+// Two bf16 -> two fp16 of the values times 2^-8 (one f32x2 multiply).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x) {
-  const float lo = __uint_as_float(x << 16) * kPfVScale;
-  const float hi = __uint_as_float(x & 0xFFFF0000u) * kPfVScale;
+  float lo, hi;
+  f2_split(f2_mul(f2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u)),
+                  f2(kPfVScale, kPfVScale)),
+           lo, hi);
   return pack2<true>(lo, hi);
 }
 
@@ -388,24 +390,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int vs = j % NV;
       if (!tc_wait(bar_v_full + 8u * vs, (j / NV) & 1, s_abort)) break;
       const uint32_t vst = sv + vs * TP::kTileBytes;
-      const bool ztile = j == zero_tile;
+      if (j != zero_tile) {
 #pragma unroll 4
-      for (int i = 0; i < kChunks; ++i) {
-        const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
-        uint4 v;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(vst + off));
-        const int key = static_cast<int>((off % TP::kKVHalfBytes) >> 7);
-        if (ztile && (key >> 4) == zero_blk && (key & 15) >= tail) {
-          v = make_uint4(0u, 0u, 0u, 0u);
-        } else {
+        for (int i = 0; i < kChunks; ++i) {
+          const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(vst + off));
           v.x = bf16x2_to_f16x2_scaled(v.x);
           v.y = bf16x2_to_f16x2_scaled(v.y);
           v.z = bf16x2_to_f16x2_scaled(v.z);
           v.w = bf16x2_to_f16x2_scaled(v.w);
+          st_shared_v4(vst + off, v);
         }
-        st_shared_v4(vst + off, v);
+      } else {
+        // the tile holding the context's last, partly filled block: its rows
+        // past the context end become zeros
+        for (int i = 0; i < kChunks; ++i) {
+          const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(vst + off));
+          const int key = static_cast<int>((off % TP::kKVHalfBytes) >> 7);
+          if ((key >> 4) == zero_blk && (key & 15) >= tail) {
+            v = make_uint4(0u, 0u, 0u, 0u);
+          } else {
+            v.x = bf16x2_to_f16x2_scaled(v.x);
+            v.y = bf16x2_to_f16x2_scaled(v.y);
+            v.z = bf16x2_to_f16x2_scaled(v.z);
+            v.w = bf16x2_to_f16x2_scaled(v.w);
+          }
+          st_shared_v4(vst + off, v);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_v_conv + 8u * vs);
