@@ -34,10 +34,14 @@
 //   * warps 0-3 / 4-7 (softmax of query tile 0 / 1): thread (warp w) owns
 //     row 32 (w % 4) + lane of its tile (its tensor-memory lane). It reads
 //     the row's 128 scores, applies the scale and the causal mask, and keeps
-//     a running max m and sum l in the exp2 domain. The max used for P is
-//     only raised when a row's tile max exceeds it by more than 2^8 (then
-//     O's row is rescaled in tensor memory; PV_g(j-1) has completed once
-//     S_g(j) has), so P <= 2^8. The arguments are formed with f32x2 FMAs,
+//     a running reference m and sum l in the exp2 domain. A tile with masked
+//     keys, or a row's first, takes its max first and raises m only when the
+//     tile max exceeds it by more than 2^8 (then O's row is rescaled in
+//     tensor memory; PV_g(j-1) has completed once S_g(j) has), so P <= 2^8
+//     there. Any other tile is formed against m as it stands, with no max
+//     at all, and kept if its P sum is at most 2^15 (so is every P, inside
+//     fp16's range); otherwise it is redone max first. The arguments are
+//     formed with f32x2 FMAs,
 //     P is rounded to fp16 (11 significant bits) and written over the first
 //     64 score columns, and l sums P in fp32 (f32x2 adds) before rounding.
 //     At the end each thread scales its O row by 2^8 / l; a tile whose
@@ -71,6 +75,7 @@ constexpr int kPfOtherRegs = 64;                //   + 2 x 128 x 64 = 512 x 128
 static_assert(kPfSoftmaxRegs + kPfOtherRegs == 2 * (65536 / kPfThreads),
               "register split must add up to the launch's registers");
 constexpr float kPfRescaleLog2 = 8.f;           // raise the max only past 2^8
+constexpr float kPfSpecSumMax = 32768.f;        // a speculative tile's P sums to <= 2^15
 constexpr float kPfVScale = 1.f / 256.f;        // V widened to fp16 as v * 2^-8
 constexpr float kPfOutScale = 256.f;
 
@@ -463,16 +468,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const bool open = __all_sync(0xffffffffu, kb + kPfKeys - 1 <= klim);
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
       // An open tile after the row's first one is taken speculatively: P
-      // is formed against the max already in use while the tile's largest
-      // argument is tracked beside it, so the exponentials (the special-
-      // function unit) do not wait for a max reduction. Only if some row's
-      // largest argument exceeds 2^8 (the max must be raised) is the tile
-      // redone the plain way, which computes the same P as the speculative
-      // pass wherever the max stays.
+      // is formed against the max already in use, with no max reduction at
+      // all. The softmax is the same for any reference m, so the only risk
+      // is range: if the tile's sum of P stays at most 2^15, every P does,
+      // and fp16 (largest finite 65504) holds it with its usual relative
+      // precision. Only a tile whose sum exceeds that (or is not finite) is
+      // redone the plain way, with the max raised to the tile's.
       bool redo = true;
       if (open && __all_sync(0xffffffffu, m_used != -INFINITY)) {
         const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_used, -m_used);
-        float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pk[32];
@@ -481,15 +485,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int c = 64 * hh + 2 * e;
             float x0, x1;
             f2_split(f2_fma(f2(z[c], z[c + 1]), sc2, nm2), x0, x1);
-            xm[e & 3] = fmax3(xm[e & 3], x0, x1);
             const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             pk[e] = pack2<true>(p0, p1);
             lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
           }
           tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
         }
-        redo = __any_sync(0xffffffffu,
-                          fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3])) > kPfRescaleLog2);
+        float a0, a1, b0, b1;
+        f2_split(lsum[0], a0, a1);
+        f2_split(lsum[1], b0, b1);
+        redo = __any_sync(0xffffffffu, !((a0 + b0) + (a1 + b1) <= kPfSpecSumMax));
         if (redo) {
           tc_wait_st();  // the plain pass rewrites the same columns
           lsum[0] = lsum[1] = f2(0.f, 0.f);
