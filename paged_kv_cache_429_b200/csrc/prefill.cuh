@@ -467,16 +467,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // row without a visible key (the warp takes this branch as one)
       const bool open = __all_sync(0xffffffffu, kb + kPfKeys - 1 <= klim);
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-      // An open tile after the row's first one is taken speculatively: P
-      // is formed against the max already in use, with no max reduction at
-      // all. The softmax is the same for any reference m, so the only risk
-      // is range: if the tile's sum of P stays at most 2^15, every P does,
-      // and fp16 (largest finite 65504) holds it with its usual relative
-      // precision. Only a tile whose sum exceeds that (or is not finite) is
-      // redone the plain way, with the max raised to the tile's.
-      bool redo = true;
-      if (open && __all_sync(0xffffffffu, m_used != -INFINITY)) {
-        const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_used, -m_used);
+      // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
+      // over the first 64 score columns; l sums P in fp32 before rounding.
+      // The pairs' arguments come from one f32x2 FMA against -m (-inf for a
+      // row with no visible key yet, whose P is then 0); each half of 64
+      // keys (32 columns) is stored as soon as it is packed, its scores
+      // already in registers.
+      auto form_p = [&](float neg_m) {
+        const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t pk[32];
@@ -491,6 +489,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
         }
+      };
+      // An open tile after the row's first one is taken speculatively: P
+      // is formed against the max already in use, with no max reduction at
+      // all. The softmax is the same for any reference m, so the only risk
+      // is range: if the tile's sum of P stays at most 2^15, every P does,
+      // and fp16 (largest finite 65504) holds it with its usual relative
+      // precision. Only a tile whose sum exceeds that (or is not finite) is
+      // redone the plain way, with the max raised to the tile's.
+      bool redo = true;
+      if (open && __all_sync(0xffffffffu, m_used != -INFINITY)) {
+        form_p(-m_used);
         float a0, a1, b0, b1;
         f2_split(lsum[0], a0, a1);
         f2_split(lsum[1], b0, b1);
@@ -501,6 +510,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       if (redo) {
+        // masked keys (NaN allowed past the context end) become -inf
         if (!open && kb + kPfKeys - 1 > klim) {
 #pragma unroll
           for (int c = 0; c < kPfKeys; ++c)
@@ -523,42 +533,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
         l *= alpha;
         m_used = m_new;
-        // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
-        // over the first 64 score columns; l sums P in fp32 before
-        // rounding. Open tiles form the pairs' arguments with one f32x2
-        // FMA; tiles with masked keys or dead rows go element by element
-        // and zero dead rows. Each half of 64 keys (32 columns) is stored
-        // as soon as it is packed: its scores are already in registers.
-        const bool live = valid && m_used != -INFINITY;
-        const float neg_m = -m_used;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
-          if (open) {
-            const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = 64 * hh + 2 * e;
-              const uint64_t x = f2_fma(f2(z[c], z[c + 1]), sc2, nm2);
-              float p0, p1;
-              f2_split(x, p0, p1);
-              p0 = ex2_approx(p0);
-              p1 = ex2_approx(p1);
-              pk[e] = pack2<true>(p0, p1);
-              lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = 64 * hh + 2 * e;
-              const float p0 = live ? ex2_approx(fmaf(z[c], scale, neg_m)) : 0.f;
-              const float p1 = live ? ex2_approx(fmaf(z[c + 1], scale, neg_m)) : 0.f;
-              pk[e] = pack2<true>(p0, p1);
-              lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
-            }
-          }
-          tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
-        }
+        form_p(m_used == -INFINITY ? -INFINITY : -m_used);
         if (j > 0 && __any_sync(0xffffffffu, raise)) {
           // O_g holds PV_g(j-1): it completed before S_g(j)
 #pragma unroll
