@@ -34,14 +34,14 @@
 //   * warps 0-3 / 4-7 (softmax of query tile 0 / 1): thread (warp w) owns
 //     row 32 (w % 4) + lane of its tile (its tensor-memory lane). It reads
 //     the row's 128 scores, applies the scale and the causal mask, and keeps
-//     a running reference m and sum l in the exp2 domain. A tile with masked
-//     keys, or a row's first, takes its max first and raises m only when the
-//     tile max exceeds it by more than 2^8 (then O's row is rescaled in
-//     tensor memory; PV_g(j-1) has completed once S_g(j) has), so P <= 2^8
-//     there. Any other tile is formed against m as it stands, with no max
-//     at all, and kept if its P sum is at most 2^15 (so is every P, inside
-//     fp16's range); otherwise it is redone max first. The arguments are
-//     formed with f32x2 FMAs,
+//     a running reference m and sum l in the exp2 domain. A row's first
+//     tile takes its max first and raises m only when the tile max exceeds
+//     it by more than 2^8 (then O's row is rescaled in tensor memory;
+//     PV_g(j-1) has completed once S_g(j) has), so P <= 2^8 there. Any
+//     other tile is formed against m as it stands, with no max at all, and
+//     kept if its P sum is at most 2^15 (so is every P, inside fp16's
+//     range); otherwise it is redone max first. The arguments are formed
+//     with f32x2 FMAs,
 //     P is rounded to fp16 (11 significant bits) and written over the first
 //     64 score columns, and l sums P in fp32 (f32x2 adds) before rounding.
 //     At the end each thread scales its O row by 2^8 / l; a tile whose
@@ -463,9 +463,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
       for (int c = 0; c < kPfKeys; ++c) z[c] = __uint_as_float(sr[c >> 5][c & 31]);
       const int kb = j * kPfKeys;
-      // every row of the warp sees every key of the tile: no mask, and no
-      // row without a visible key (the warp takes this branch as one)
-      const bool open = __all_sync(0xffffffffu, kb + kPfKeys - 1 <= klim);
+      // masked keys (NaN allowed past the context end) become -inf
+      if (kb + kPfKeys - 1 > klim) {
+#pragma unroll
+        for (int c = 0; c < kPfKeys; ++c)
+          if (kb + c > klim) z[c] = -INFINITY;
+      }
       uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
       // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
       // over the first 64 score columns; l sums P in fp32 before rounding.
@@ -490,32 +493,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
         }
       };
-      // An open tile after the row's first one is taken speculatively: P
-      // is formed against the max already in use, with no max reduction at
-      // all. The softmax is the same for any reference m, so the only risk
-      // is range: if the tile's sum of P stays at most 2^15, every P does,
-      // and fp16 (largest finite 65504) holds it with its usual relative
-      // precision. Only a tile whose sum exceeds that (or is not finite) is
-      // redone the plain way, with the max raised to the tile's.
+      // A tile after a row's first one is taken speculatively: P is formed
+      // against the reference already in use (the max of earlier tiles), with
+      // no max reduction at all. The softmax is the same for any reference,
+      // so the only risk is range: if the tile's sum of P stays at most 2^15,
+      // every P does, and fp16 (largest finite 65504) holds it with its
+      // usual relative precision. A row's first tile, and a tile whose sum
+      // is out of range or not finite, is done max first (the reference
+      // raised to the tile's max), so each row's largest weight is exact.
+      // Rows outside the chunk have every key masked and P = 0 either way.
       bool redo = true;
-      if (open && __all_sync(0xffffffffu, m_used != -INFINITY)) {
-        form_p(-m_used);
+      if (__all_sync(0xffffffffu, !valid || m_used != -INFINITY)) {
+        form_p(m_used == -INFINITY ? -INFINITY : -m_used);
         float a0, a1, b0, b1;
         f2_split(lsum[0], a0, a1);
         f2_split(lsum[1], b0, b1);
-        redo = __any_sync(0xffffffffu, !((a0 + b0) + (a1 + b1) <= kPfSpecSumMax));
+        redo = __any_sync(0xffffffffu, valid && !((a0 + b0) + (a1 + b1) <= kPfSpecSumMax));
         if (redo) {
-          tc_wait_st();  // the plain pass rewrites the same columns
+          tc_wait_st();  // the max-first pass rewrites the same columns
           lsum[0] = lsum[1] = f2(0.f, 0.f);
         }
       }
       if (redo) {
-        // masked keys (NaN allowed past the context end) become -inf
-        if (!open && kb + kPfKeys - 1 > klim) {
-#pragma unroll
-          for (int c = 0; c < kPfKeys; ++c)
-            if (kb + c > klim) z[c] = -INFINITY;
-        }
         // tile max of the raw scores (scale > 0) as a tree of 3-input maxima
         float mx[8];
 #pragma unroll
