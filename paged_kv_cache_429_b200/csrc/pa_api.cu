@@ -474,7 +474,8 @@ pa_status pa_prefill(float *out, const void *q, const void *k_cache, const void 
   const int64_t cta_tokens = static_cast<int64_t>(pa::kPfQTiles) * p.tokens_per_tile;
   const int64_t tiles = (static_cast<int64_t>(max_query_len) + cta_tokens - 1) / cta_tokens;
   if (tiles > INT32_MAX) return PA_ERR_UNSUPPORTED;
-  dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
+  // each CTA takes two tile pairs of a chunk, a heavy and a light one
+  dim3 grid(static_cast<unsigned>((tiles + 1) / 2), num_kv_heads, num_seqs);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUtensorMap tq, tk, tv, to;
   if (!make_q_tmap(&tq, q, num_tokens, num_q_heads, head_dim, group, p.tokens_per_tile) ||

@@ -106,10 +106,12 @@ struct PfPlan {
   static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int kKOff = kPfQTiles * kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
-  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_conv[NV], v_empty[NV],
-  // s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kKStages + 3 * kVStages + 3 * kPfQTiles + 1;
+  static constexpr int kBoxBytes = kPfRows * 128;        // 32 fp32 columns of a tile's rows
+  static constexpr int kStageOff = kVOff + kVStages * kTileBytes;  // one box per query tile
+  static constexpr int kBarOff = kStageOff + kPfQTiles * kBoxBytes;
+  // q_full[2], q_free[2], k_full[NK], k_empty[NK], v_full[NV], v_conv[NV],
+  // v_empty[NV], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 2 * kKStages + 3 * kVStages + 5 * kPfQTiles + 1;
   static constexpr int kSmemBytes = 1024 + kBarOff + 8 * kNumBars + 16;
   static constexpr int kTmemCols = 512;
   static constexpr int kOCol = kPfQTiles * kPfKeys;        // O_g at kOCol + g * D
@@ -139,6 +141,27 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t x) {
   return pack2<true>(lo, hi);
 }
 
+// Work item: query tiles (2 qt, 2 qt + 1) of one (sequence, KV head) chunk,
+// tpt tokens each; what every role needs to know of it.
+struct PfItem {
+  int t0;       // first chunk token of the item
+  int nt[2];    // key tiles each query tile needs (0: the tile has no token)
+  int ntiles;   // key tiles the item streams
+  int nblk;     // cache blocks it reads
+};
+
+__device__ __forceinline__ PfItem pf_item(int qt, int n, int ctx0, int tpt) {
+  PfItem it;
+  it.t0 = qt * kPfQTiles * tpt;
+  const bool has1 = it.t0 + tpt < n;
+  // keys up to each tile's last token's position
+  it.nt[0] = (ctx0 + min(n, it.t0 + tpt) - 1) / kPfKeys + 1;
+  it.nt[1] = has1 ? (ctx0 + min(n, it.t0 + 2 * tpt) - 1) / kPfKeys + 1 : 0;
+  it.ntiles = has1 ? it.nt[1] : it.nt[0];
+  it.nblk = (ctx0 + min(n, it.t0 + kPfQTiles * tpt) - 1) / kBS + 1;
+  return it;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -158,8 +181,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t sq = base;                        // Q of tile g, half x: sq + g kQBytes + x kQHalfBytes
   const uint32_t sk = base + TP::kKOff;            // K stage st at sk + st * kTileBytes
   const uint32_t sv = base + TP::kVOff;            // V stage st at sv + st * kTileBytes
-  const uint32_t bar_q = base + TP::kBarOff;
-  const uint32_t bar_k_full = bar_q + 8;
+  const uint32_t sstage = base + TP::kStageOff;    // tile g's output staging: sstage + g kBoxBytes
+  const uint32_t bar_q = base + TP::kBarOff;                   // [tile]
+  const uint32_t bar_q_free = bar_q + 8 * kPfQTiles;           // [tile]
+  const uint32_t bar_k_full = bar_q_free + 8 * kPfQTiles;
   const uint32_t bar_k_empty = bar_k_full + 8 * NK;
   const uint32_t bar_v_full = bar_k_empty + 8 * NK;
   const uint32_t bar_v_conv = bar_v_full + 8 * NV;
@@ -171,7 +196,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(base_ptr + TP::kBarOff + 8 * TP::kNumBars);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
-  const int qt = blockIdx.x;
+  const int x = blockIdx.x;
   const int h = blockIdx.y;
   const int s = blockIdx.z;
   const int warp = threadIdx.x >> 5;
@@ -182,21 +207,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int q0 = p.query_start[s];
   const int n = min(p.query_start[s + 1] - q0, L);  // chunk length
   const int tpt = p.tokens_per_tile;
-  const int t0 = qt * kPfQTiles * tpt;              // first chunk token of this CTA
-  if (t0 >= n) return;
-  if (bad_len && threadIdx.x == 0 && qt == 0) raise_error(kErrContextClamp);
+  // Work items of this chunk: tile pairs qt = 0 .. QT-1, their causal cost
+  // growing with qt. CTA x takes qt = QT-1-x, then qt = x: every CTA but a
+  // middle one gets the same work, and the second item's first loads and
+  // the first item's output write overlap the other item's tiles.
+  const int QT = (n + kPfQTiles * tpt - 1) / (kPfQTiles * tpt);
+  if (x >= (QT + 1) / 2) return;
+  if (bad_len && threadIdx.x == 0 && x == 0) raise_error(kErrContextClamp);
+  const int nitems = (QT - 1 - x > x) ? 2 : 1;
   const int group = p.group;
   const int ctx0 = L - n;                           // position of chunk token 0
-  const bool has1 = t0 + tpt < n;                   // query tile 1 has tokens
-  // key tiles each query tile needs (keys up to its last token's position)
-  const int nt0 = (ctx0 + min(n, t0 + tpt) - 1) / kPfKeys + 1;
-  const int nt1 = has1 ? (ctx0 + min(n, t0 + 2 * tpt) - 1) / kPfKeys + 1 : 0;
-  const int ntiles = has1 ? nt1 : nt0;              // key tiles the CTA streams
-  const int kmax = ctx0 + min(n, t0 + kPfQTiles * tpt) - 1;
-  const int nblk = kmax / kBS + 1;
+  // item it: the heavier tile pair first
+  auto item = [&](int it) { return pf_item(it == 0 ? QT - 1 - x : x, n, ctx0, tpt); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    for (int g = 0; g < kPfQTiles; ++g) {
+      mbar_init(bar_q + 8u * g, 1);
+      mbar_init(bar_q_free + 8u * g, 1);
+      mbar_init(bar_s_full + 8u * g, 1);
+      mbar_init(bar_p_full + 8u * g, 4 * 32);
+      mbar_init(bar_o_done + 8u * g, 1);
+    }
     for (int i = 0; i < NK; ++i) {
       mbar_init(bar_k_full + 8u * i, 1);
       mbar_init(bar_k_empty + 8u * i, 1);
@@ -205,11 +236,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(bar_v_full + 8u * i, 1);
       mbar_init(bar_v_conv + 8u * i, 4 * 32);
       mbar_init(bar_v_empty + 8u * i, 1);
-    }
-    for (int g = 0; g < kPfQTiles; ++g) {
-      mbar_init(bar_s_full + 8u * g, 1);
-      mbar_init(bar_p_full + 8u * g, 4 * 32);
-      mbar_init(bar_o_done + 8u * g, 1);
     }
     mbar_init(bar_drain, 1);
     *s_abort = 0;
@@ -228,6 +254,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
     if (warp == kPfKWarp || warp == kPfVWarp) {
       // -------------------------------------------------------- producers
+      // warp kPfKWarp: each item's Q rows (tile g's buffer reloaded once the
+      // previous item's last score MMA of that tile has completed), then its
+      // K tiles; warp kPfVWarp: the V tiles. Both rings run on the tile
+      // count over the items.
       const bool is_k = warp == kPfKWarp;
       const int nst = is_k ? NK : NV;
       const uint32_t ring = is_k ? sk : sv;
@@ -236,61 +266,74 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const CUtensorMap *tmap = is_k ? &tmap_k : &tmap_v;
       if (lane == 0) {
         prefetch_tmap(tmap);
-        if (is_k) {
-          prefetch_tmap(&tmap_q);
-          mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * H * 128 * group * tpt);
-          for (int g = 0; g < (has1 ? 2 : 1); ++g)
-#pragma unroll
-            for (int x = 0; x < H; ++x)
-              tma_load_3d(sq + g * TP::kQBytes + x * TP::kQHalfBytes, &tmap_q, bar_q, 64 * x,
-                          h * group, q0 + t0 + g * tpt);
-        }
+        if (is_k) prefetch_tmap(&tmap_q);
       }
       const int32_t *bt = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq;
       const int total_rows = p.num_blocks * p.num_kv_heads * kBS;
       bool ok = true, bad_id = false;
-      int issued = 0;
-      int mine = -1;
-      for (int j = 0; j < ntiles && ok; ++j) {
-        // 32 table entries (4 tiles) per warp load
-        if ((j & 3) == 0) {
-          const int jb = j * kPfBlocks + lane;
-          mine = jb < nblk ? bt[jb] : -1;
-        }
-        int phys[kPfBlocks];
+      int issued = 0, G = 0;
+      int qloads[kPfQTiles] = {0, 0};
+      for (int it = 0; it < nitems && ok; ++it) {
+        const PfItem w = item(it);
+        if (is_k && lane == 0) {
+          for (int g = 0; g < kPfQTiles && ok; ++g) {
+            if (w.nt[g] == 0) continue;
+            if (qloads[g] > 0) ok = tc_wait(bar_q_free + 8u * g, (qloads[g] - 1) & 1, s_abort);
+            if (!ok) break;
+            mbar_arrive_expect_tx(bar_q + 8u * g, H * 128 * group * tpt);
 #pragma unroll
-        for (int b = 0; b < kPfBlocks; ++b)
-          phys[b] = __shfl_sync(0xffffffffu, mine, (j & 3) * kPfBlocks + b);
-        if (lane == 0) {
-          const int st = j % nst;
-          if (j >= nst) ok = tc_wait(bar_empty + 8u * st, ((j / nst) - 1) & 1, s_abort);
-          if (ok) {
-            const uint32_t full = bar_full + 8u * st;
-            const uint32_t dst = ring + st * TP::kTileBytes;
-            mbar_arrive_expect_tx(full, TP::kTileBytes);
-#pragma unroll
-            for (int b = 0; b < kPfBlocks; ++b) {
-              const bool real = j * kPfBlocks + b < nblk;
-              int y;
-              if (!real || phys[b] < 0 || phys[b] >= p.num_blocks) {
-                y = total_rows;  // past the tensor's end: TMA fills zeros
-                bad_id |= real;
-              } else {
-                y = (phys[b] * p.num_kv_heads + h) * kBS;
-              }
-#pragma unroll
-              for (int x = 0; x < H; ++x)
-                tma_load_2d(dst + x * TP::kKVHalfBytes + b * 2048, tmap, full, 64 * x, y);
-            }
-            issued = j + 1;
+            for (int xx = 0; xx < H; ++xx)
+              tma_load_3d(sq + g * TP::kQBytes + xx * TP::kQHalfBytes, &tmap_q, bar_q + 8u * g,
+                          64 * xx, h * group, q0 + w.t0 + g * tpt);
+            ++qloads[g];
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
+        int mine = -1;
+        for (int j = 0; j < w.ntiles && ok; ++j) {
+          // 32 table entries (4 tiles) per warp load
+          if ((j & 3) == 0) {
+            const int jb = j * kPfBlocks + lane;
+            mine = jb < w.nblk ? bt[jb] : -1;
+          }
+          int phys[kPfBlocks];
+#pragma unroll
+          for (int b = 0; b < kPfBlocks; ++b)
+            phys[b] = __shfl_sync(0xffffffffu, mine, (j & 3) * kPfBlocks + b);
+          if (lane == 0) {
+            const int st = G % nst;
+            if (G >= nst) ok = tc_wait(bar_empty + 8u * st, ((G / nst) - 1) & 1, s_abort);
+            if (ok) {
+              const uint32_t full = bar_full + 8u * st;
+              const uint32_t dst = ring + st * TP::kTileBytes;
+              mbar_arrive_expect_tx(full, TP::kTileBytes);
+#pragma unroll
+              for (int b = 0; b < kPfBlocks; ++b) {
+                const bool real = j * kPfBlocks + b < w.nblk;
+                int y;
+                if (!real || phys[b] < 0 || phys[b] >= p.num_blocks) {
+                  y = total_rows;  // past the tensor's end: TMA fills zeros
+                  bad_id |= real;
+                } else {
+                  y = (phys[b] * p.num_kv_heads + h) * kBS;
+                }
+#pragma unroll
+                for (int xx = 0; xx < H; ++xx)
+                  tma_load_2d(dst + xx * TP::kKVHalfBytes + b * 2048, tmap, full, 64 * xx, y);
+              }
+              issued = G + 1;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ++G;
+        }
       }
       if (lane == 0) {
         if (bad_id && is_k) raise_error(kErrBlockRange);
         // no bulk copy may still be landing when the CTA exits
-        if (is_k) mbar_wait_bounded(bar_q, 0, kWaitLimitNs);
+        if (is_k)
+          for (int g = 0; g < kPfQTiles; ++g)
+            if (qloads[g] > 0) mbar_wait_bounded(bar_q + 8u * g, (qloads[g] - 1) & 1, kWaitLimitNs);
         for (int j = max(0, issued - nst); j < issued; ++j)
           mbar_wait_bounded(bar_full + 8u * (j % nst), (j / nst) & 1, kWaitLimitNs);
       }
@@ -299,10 +342,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (lane == 0) {
         constexpr uint32_t id_s = tc_idesc_bf16(kPfRows, kPfKeys, false);
         constexpr uint32_t id_pv = tc_idesc_f16(kPfRows, D, true);
-        bool ok = tc_wait(bar_q, 0, s_abort);
-        auto wait_k = [&](int j) -> uint32_t {
-          const int st = j % NK;
-          ok = ok && tc_wait(bar_k_full + 8u * st, (j / NK) & 1, s_abort);
+        bool ok = true;
+        int G = 0;                      // K/V tiles of earlier items
+        int cnt[kPfQTiles] = {0, 0};    // P of each query tile consumed so far
+        int qph[kPfQTiles] = {0, 0};    // Q loads of each tile consumed so far
+        auto wait_k = [&](int gi) -> uint32_t {
+          const int st = gi % NK;
+          ok = ok && tc_wait(bar_k_full + 8u * st, (gi / NK) & 1, s_abort);
           tc_fence_after_sync();
           return sk + st * TP::kTileBytes;
         };
@@ -320,7 +366,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_commit(bar_s_full + 8u * g);
         };
         // O_g += P_g V: P_g (fp16, 16 keys per 8 columns) in the first 64 of
-        // tile g's score columns, V fp16 in shared memory, 16 keys per MMA
+        // tile g's score columns, V fp16 in shared memory, 16 keys per MMA;
+        // the item's first key tile overwrites O_g
         auto issue_pv = [&](int g, uint32_t vst, int j) {
           const uint32_t pt = tmem + g * kPfKeys;
           const uint32_t o = tmem + TP::kOCol + g * D;
@@ -331,47 +378,79 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const uint64_t b = tc_desc_sw128(vst + kk * 2048, TP::kKVHalfBytes, 1024);
             tc_mma_ts(o, pt + kk * 8, b, id_pv, j > 0 || kk > 0);
           }
-          if (j == (g == 0 ? nt0 : nt1) - 1) tc_commit(bar_o_done + 8u * g);
         };
-        if (ok) {
-          const uint32_t kst = wait_k(0);
-          if (ok) {
-            issue_s(0, kst);
-            if (nt1 > 0) issue_s(1, kst);
-            tc_commit(bar_k_empty);
-          }
-        }
-        for (int j = 0; j < ntiles && ok; ++j) {
-          const int vs = j % NV;
-          const uint32_t vst = sv + vs * TP::kTileBytes;
-          bool v_ready = false;
-          if (j < nt0) {
-            ok = tc_wait(bar_p_full, j & 1, s_abort) &&
-                 tc_wait(bar_v_conv + 8u * vs, (j / NV) & 1, s_abort);
+        for (int it = 0; it < nitems && ok; ++it) {
+          const PfItem w = item(it);
+          // the next item reloads tile g's Q once this item's last S_g is done
+          bool q_next[kPfQTiles];
+#pragma unroll
+          for (int g = 0; g < kPfQTiles; ++g)
+            q_next[g] = it + 1 < nitems && item(it + 1).nt[g] > 0 && w.nt[g] > 0;
+#pragma unroll
+          for (int g = 0; g < kPfQTiles; ++g)
+            if (w.nt[g] > 0) {
+              ok = ok && tc_wait(bar_q + 8u * g, qph[g] & 1, s_abort);
+              ++qph[g];
+            }
+          if (!ok) break;
+          {
+            const uint32_t kst = wait_k(G);
             if (!ok) break;
-            v_ready = true;
-            tc_fence_after_sync();
-            issue_pv(0, vst, j);
+#pragma unroll
+            for (int g = 0; g < kPfQTiles; ++g)
+              if (w.nt[g] > 0) {
+                issue_s(g, kst);
+                if (w.nt[g] == 1 && q_next[g]) tc_commit(bar_q_free + 8u * g);
+              }
+            tc_commit(bar_k_empty + 8u * (G % NK));
           }
-          const bool knext = j + 1 < ntiles;
-          uint32_t kst = 0;
-          if (knext) {
-            kst = wait_k(j + 1);
-            if (!ok) break;
-            if (j + 1 < nt0) issue_s(0, kst);
+          // Per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1); S_g(j+1)
+          // overwrites the columns P_g(j) is read from and is issued after
+          // PV_g(j) (one thread's MMAs run in issue order).
+          for (int j = 0; j < w.ntiles && ok; ++j) {
+            const int gv = G + j;
+            const int vs = gv % NV;
+            const uint32_t vst = sv + vs * TP::kTileBytes;
+            bool v_ready = false;
+            if (j < w.nt[0]) {
+              ok = tc_wait(bar_p_full, cnt[0] & 1, s_abort) &&
+                   tc_wait(bar_v_conv + 8u * vs, (gv / NV) & 1, s_abort);
+              if (!ok) break;
+              ++cnt[0];
+              v_ready = true;
+              tc_fence_after_sync();
+              issue_pv(0, vst, j);
+              if (j == w.nt[0] - 1) tc_commit(bar_o_done);
+            }
+            const bool knext = j + 1 < w.ntiles;
+            uint32_t kst = 0;
+            if (knext) {
+              kst = wait_k(gv + 1);
+              if (!ok) break;
+              if (j + 1 < w.nt[0]) {
+                issue_s(0, kst);
+                if (j + 2 == w.nt[0] && q_next[0]) tc_commit(bar_q_free);
+              }
+            }
+            if (j < w.nt[1]) {
+              ok = tc_wait(bar_p_full + 8u, cnt[1] & 1, s_abort) &&
+                   (v_ready || tc_wait(bar_v_conv + 8u * vs, (gv / NV) & 1, s_abort));
+              if (!ok) break;
+              ++cnt[1];
+              tc_fence_after_sync();
+              issue_pv(1, vst, j);
+              if (j == w.nt[1] - 1) tc_commit(bar_o_done + 8u);
+            }
+            tc_commit(bar_v_empty + 8u * vs);
+            if (knext) {
+              if (j + 1 < w.nt[1]) {
+                issue_s(1, kst);
+                if (j + 2 == w.nt[1] && q_next[1]) tc_commit(bar_q_free + 8u);
+              }
+              tc_commit(bar_k_empty + 8u * ((gv + 1) % NK));
+            }
           }
-          if (j < nt1) {
-            ok = tc_wait(bar_p_full + 8u, j & 1, s_abort) &&
-                 (v_ready || tc_wait(bar_v_conv + 8u * vs, (j / NV) & 1, s_abort));
-            if (!ok) break;
-            tc_fence_after_sync();
-            issue_pv(1, vst, j);
-          }
-          tc_commit(bar_v_empty + 8u * vs);
-          if (knext) {
-            if (j + 1 < nt1) issue_s(1, kst);
-            tc_commit(bar_k_empty + 8u * ((j + 1) % NK));
-          }
+          G += w.ntiles;
         }
         // every MMA issued here has completed before tensor memory is freed
         tc_commit(bar_drain);
@@ -388,50 +467,61 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int c = threadIdx.x - kPfCvtWarp0 * 32;
     const int tail = L % kBS;
     const int last_blk = (L - 1) / kBS;
-    const int zero_tile = (tail != 0 && last_blk < nblk) ? last_blk / kPfBlocks : -1;
     const int zero_blk = last_blk % kPfBlocks;
     constexpr int kChunks = TP::kTileBytes / 16 / 128;
-    for (int j = 0; j < ntiles; ++j) {
-      const int vs = j % NV;
-      if (!tc_wait(bar_v_full + 8u * vs, (j / NV) & 1, s_abort)) break;
-      const uint32_t vst = sv + vs * TP::kTileBytes;
-      if (j != zero_tile) {
-#pragma unroll 4
-        for (int i = 0; i < kChunks; ++i) {
-          const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
-          uint4 v;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(vst + off));
-          v.x = bf16x2_to_f16x2_scaled(v.x);
-          v.y = bf16x2_to_f16x2_scaled(v.y);
-          v.z = bf16x2_to_f16x2_scaled(v.z);
-          v.w = bf16x2_to_f16x2_scaled(v.w);
-          st_shared_v4(vst + off, v);
+    int G = 0;
+    for (int it = 0; it < nitems; ++it) {
+      const PfItem w = item(it);
+      const int zero_tile = (tail != 0 && last_blk < w.nblk) ? last_blk / kPfBlocks : -1;
+      bool ok = true;
+      for (int j = 0; j < w.ntiles; ++j) {
+        const int gv = G + j;
+        const int vs = gv % NV;
+        if (!tc_wait(bar_v_full + 8u * vs, (gv / NV) & 1, s_abort)) {
+          ok = false;
+          break;
         }
-      } else {
-        // the tile holding the context's last, partly filled block: its rows
-        // past the context end become zeros
-        for (int i = 0; i < kChunks; ++i) {
-          const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
-          uint4 v;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(vst + off));
-          const int key = static_cast<int>((off % TP::kKVHalfBytes) >> 7);
-          if ((key >> 4) == zero_blk && (key & 15) >= tail) {
-            v = make_uint4(0u, 0u, 0u, 0u);
-          } else {
+        const uint32_t vst = sv + vs * TP::kTileBytes;
+        if (j != zero_tile) {
+#pragma unroll 4
+          for (int i = 0; i < kChunks; ++i) {
+            const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(vst + off));
             v.x = bf16x2_to_f16x2_scaled(v.x);
             v.y = bf16x2_to_f16x2_scaled(v.y);
             v.z = bf16x2_to_f16x2_scaled(v.z);
             v.w = bf16x2_to_f16x2_scaled(v.w);
+            st_shared_v4(vst + off, v);
           }
-          st_shared_v4(vst + off, v);
+        } else {
+          // the tile holding the context's last, partly filled block: its
+          // rows past the context end become zeros
+          for (int i = 0; i < kChunks; ++i) {
+            const uint32_t off = static_cast<uint32_t>(i * 128 + c) * 16u;
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(vst + off));
+            const int key = static_cast<int>((off % TP::kKVHalfBytes) >> 7);
+            if ((key >> 4) == zero_blk && (key & 15) >= tail) {
+              v = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+              v.x = bf16x2_to_f16x2_scaled(v.x);
+              v.y = bf16x2_to_f16x2_scaled(v.y);
+              v.z = bf16x2_to_f16x2_scaled(v.z);
+              v.w = bf16x2_to_f16x2_scaled(v.w);
+            }
+            st_shared_v4(vst + off, v);
+          }
         }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_v_conv + 8u * vs);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_v_conv + 8u * vs);
+      if (!ok) break;
+      G += w.ntiles;
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPfSoftmaxRegs));
@@ -441,147 +531,152 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int r = quarter * 32 + lane;            // row = tensor-memory lane
     const int tl = r / group;
     const int nh = r - tl * group;
-    const int tok = t0 + g * tpt + tl;            // chunk token of this row
-    const bool valid = tl < tpt && tok < n;
-    const int klim = valid ? ctx0 + tok : -1;     // keys <= klim are visible
-    const int ntg = g == 0 ? nt0 : nt1;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t scol = g * kPfKeys;
     const uint32_t ocol = TP::kOCol + g * D;
     const float scale = p.score_scale;
-    float m_used = -INFINITY, l = 0.f;
+    const uint32_t stage = sstage + g * TP::kBoxBytes;
     bool ok = true;
-    for (int j = 0; j < ntg; ++j) {
-      ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8u * g, j & 1, s_abort));
-      if (!ok) break;
-      tc_fence_after_sync();
-      uint32_t sr[4][32];
+    int cnt = 0;  // score tiles of this query tile over the items
+    int oph = 0;  // items in which this query tile had tokens
+    for (int it = 0; it < nitems; ++it) {
+      const PfItem w = item(it);
+      const int ntg = w.nt[g];
+      if (ntg == 0) continue;
+      const int tok = w.t0 + g * tpt + tl;          // chunk token of this row
+      const bool valid = tl < tpt && tok < n;
+      const int klim = valid ? ctx0 + tok : -1;     // keys <= klim are visible
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < ntg && ok; ++j) {
+        ok = __all_sync(0xffffffffu, tc_wait(bar_s_full + 8u * g, cnt & 1, s_abort));
+        if (!ok) break;
+        ++cnt;
+        tc_fence_after_sync();
+        uint32_t sr[4][32];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) tc_ld_32x32b_x32(trow + scol + 32 * x, sr[x]);
-      tc_wait_ld();
-      float z[kPfKeys];
+        for (int x = 0; x < 4; ++x) tc_ld_32x32b_x32(trow + scol + 32 * x, sr[x]);
+        tc_wait_ld();
+        float z[kPfKeys];
 #pragma unroll
-      for (int c = 0; c < kPfKeys; ++c) z[c] = __uint_as_float(sr[c >> 5][c & 31]);
-      const int kb = j * kPfKeys;
-      // masked keys (NaN allowed past the context end) become -inf
-      if (kb + kPfKeys - 1 > klim) {
+        for (int c = 0; c < kPfKeys; ++c) z[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        const int kb = j * kPfKeys;
+        // masked keys (NaN allowed past the context end) become -inf
+        if (kb + kPfKeys - 1 > klim) {
 #pragma unroll
-        for (int c = 0; c < kPfKeys; ++c)
-          if (kb + c > klim) z[c] = -INFINITY;
-      }
-      uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-      // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
-      // over the first 64 score columns; l sums P in fp32 before rounding.
-      // The pairs' arguments come from one f32x2 FMA against -m (-inf for a
-      // row with no visible key yet, whose P is then 0); each half of 64
-      // keys (32 columns) is stored as soon as it is packed, its scores
-      // already in registers.
-      auto form_p = [&](float neg_m) {
-        const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
+          for (int c = 0; c < kPfKeys; ++c)
+            if (kb + c > klim) z[c] = -INFINITY;
+        }
+        uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        // P = 2^(z scale - m) as fp16 pairs (the lower key in the low half)
+        // over the first 64 score columns; l sums P in fp32 before rounding.
+        // The pairs' arguments come from one f32x2 FMA against -m (-inf for a
+        // row with no visible key yet, whose P is then 0); each half of 64
+        // keys (32 columns) is stored as soon as it is packed, its scores
+        // already in registers.
+        auto form_p = [&](float neg_m) {
+          const uint64_t sc2 = f2(scale, scale), nm2 = f2(neg_m, neg_m);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[32];
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = 64 * hh + 2 * e;
-            float x0, x1;
-            f2_split(f2_fma(f2(z[c], z[c + 1]), sc2, nm2), x0, x1);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            pk[e] = pack2<true>(p0, p1);
-            lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+            for (int e = 0; e < 32; ++e) {
+              const int c = 64 * hh + 2 * e;
+              float x0, x1;
+              f2_split(f2_fma(f2(z[c], z[c + 1]), sc2, nm2), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              pk[e] = pack2<true>(p0, p1);
+              lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+            }
+            tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
           }
-          tc_st_32x32b_x32(trow + scol + 32 * hh, pk);
+        };
+        // A tile after a row's first one is taken speculatively: P is formed
+        // against the reference already in use (the max of earlier tiles), with
+        // no max reduction at all. The softmax is the same for any reference,
+        // so the only risk is range: if the tile's sum of P stays at most 2^15,
+        // every P does, and fp16 (largest finite 65504) holds it with its
+        // usual relative precision. A row's first tile, and a tile whose sum
+        // is out of range or not finite, is done max first (the reference
+        // raised to the tile's max), so each row's largest weight is exact.
+        // Rows outside the chunk have every key masked and P = 0 either way.
+        bool redo = true;
+        if (__all_sync(0xffffffffu, !valid || m_used != -INFINITY)) {
+          form_p(m_used == -INFINITY ? -INFINITY : -m_used);
+          float a0, a1, b0, b1;
+          f2_split(lsum[0], a0, a1);
+          f2_split(lsum[1], b0, b1);
+          redo = __any_sync(0xffffffffu, valid && !((a0 + b0) + (a1 + b1) <= kPfSpecSumMax));
+          if (redo) {
+            tc_wait_st();  // the max-first pass rewrites the same columns
+            lsum[0] = lsum[1] = f2(0.f, 0.f);
+          }
         }
-      };
-      // A tile after a row's first one is taken speculatively: P is formed
-      // against the reference already in use (the max of earlier tiles), with
-      // no max reduction at all. The softmax is the same for any reference,
-      // so the only risk is range: if the tile's sum of P stays at most 2^15,
-      // every P does, and fp16 (largest finite 65504) holds it with its
-      // usual relative precision. A row's first tile, and a tile whose sum
-      // is out of range or not finite, is done max first (the reference
-      // raised to the tile's max), so each row's largest weight is exact.
-      // Rows outside the chunk have every key masked and P = 0 either way.
-      bool redo = true;
-      if (__all_sync(0xffffffffu, !valid || m_used != -INFINITY)) {
-        form_p(m_used == -INFINITY ? -INFINITY : -m_used);
-        float a0, a1, b0, b1;
-        f2_split(lsum[0], a0, a1);
-        f2_split(lsum[1], b0, b1);
-        redo = __any_sync(0xffffffffu, valid && !((a0 + b0) + (a1 + b1) <= kPfSpecSumMax));
         if (redo) {
-          tc_wait_st();  // the max-first pass rewrites the same columns
-          lsum[0] = lsum[1] = f2(0.f, 0.f);
+          // tile max of the raw scores (scale > 0) as a tree of 3-input maxima
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmax3(z[i], z[i + 8], z[i + 16]);
+#pragma unroll
+          for (int c = 24; c + 16 <= kPfKeys; c += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], z[c + i], z[c + 8 + i]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[kPfKeys - 8 + i]);
+          const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7])) * scale;
+          const float m_new = (mt > m_used + kPfRescaleLog2) ? mt : m_used;
+          const bool raise = m_new != m_used;
+          const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
+          l *= alpha;
+          m_used = m_new;
+          form_p(m_used == -INFINITY ? -INFINITY : -m_used);
+          if (j > 0 && __any_sync(0xffffffffu, raise)) {
+            // O_g holds PV_g(j-1): it completed before S_g(j)
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+              tc_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tc_st_32x32b_x32(trow + ocol + cc * 32, o);
+            }
+          }
         }
+        {
+          float a0, a1, b0, b1;
+          f2_split(lsum[0], a0, a1);
+          f2_split(lsum[1], b0, b1);
+          l += (a0 + b0) + (a1 + b1);
+        }
+        tc_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar_p_full + 8u * g);
       }
-      if (redo) {
-        // tile max of the raw scores (scale > 0) as a tree of 3-input maxima
-        float mx[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(z[i], z[i + 8], z[i + 16]);
-#pragma unroll
-        for (int c = 24; c + 16 <= kPfKeys; c += 16)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], z[c + i], z[c + 8 + i]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], z[kPfKeys - 8 + i]);
-        const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                               fmaxf(mx[6], mx[7])) * scale;
-        const float m_new = (mt > m_used + kPfRescaleLog2) ? mt : m_used;
-        const bool raise = m_new != m_used;
-        const float alpha = raise ? ex2_approx(m_used - m_new) : 1.f;
-        l *= alpha;
-        m_used = m_new;
-        form_p(m_used == -INFINITY ? -INFINITY : -m_used);
-        if (j > 0 && __any_sync(0xffffffffu, raise)) {
-          // O_g holds PV_g(j-1): it completed before S_g(j)
-#pragma unroll
+      // ------------------------------------------------------------ epilogue
+      if (ok) ok = __all_sync(0xffffffffu, tc_wait(bar_o_done + 8u * g, oph & 1, s_abort));
+      ++oph;
+      // the warpgroup decides together (the staged path below has barriers
+      // over its 128 threads): every warp that reaches here votes
+      ok = named_bar_and(1 + g, 128, ok);
+      if (ok) {
+        tc_fence_after_sync();
+        const float inv = l > 0.f ? kPfOutScale / l : 0.f;
+        if (w.t0 + g * tpt + tpt <= n) {
+          // Every token of the tile is in the chunk: stage O through this
+          // tile's own buffer, one box of 32 fp32 columns x the tile's rows at
+          // a time, in the 128-byte swizzled layout (thread r writes row r, its
+          // 16-byte chunk c at c ^ (r % 8): no bank conflicts), and write it
+          // with a TMA store. The last box's store drains while the next item
+          // runs; the buffer is reused only once the store has read it.
+          const uint32_t bar_id = 1 + g;
+          const uint32_t rowp = stage + r * 128;
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
             tc_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc_st_32x32b_x32(trow + ocol + cc * 32, o);
-          }
-        }
-      }
-      {
-        float a0, a1, b0, b1;
-        f2_split(lsum[0], a0, a1);
-        f2_split(lsum[1], b0, b1);
-        l += (a0 + b0) + (a1 + b1);
-      }
-      tc_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(bar_p_full + 8u * g);
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok && ntg > 0)
-      ok = __all_sync(0xffffffffu, tc_wait(bar_o_done + 8u * g, 0, s_abort));
-    // the warpgroup decides together (the staged path below has barriers
-    // over its 128 threads): every warp that reaches here votes
-    if (ntg > 0) ok = named_bar_and(1 + g, 128, ok);
-    if (ok && ntg > 0) {
-      tc_fence_after_sync();
-      const float inv = l > 0.f ? kPfOutScale / l : 0.f;
-      if (t0 + g * tpt + tpt <= n) {
-        // Every token of the tile is in the chunk: stage O through this
-        // tile's Q buffer (all of its score MMAs have completed) as boxes of
-        // 32 fp32 columns x the tile's rows in the 128-byte swizzled layout
-        // (thread r writes row r, its 16-byte chunk c at c ^ (r % 8): no bank
-        // conflicts) and write them with TMA stores, H boxes per round.
-        const uint32_t stage = sq + g * TP::kQBytes;
-        const uint32_t bar_id = 1 + g;
-#pragma unroll
-        for (int rd = 0; rd < 2; ++rd) {
-#pragma unroll
-          for (int bx = 0; bx < H; ++bx) {
-            const int cc = rd * H + bx;  // 32-column block
-            uint32_t o[32];
-            tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
-            tc_wait_ld();
-            const uint32_t rowp = stage + bx * (kPfRows * 128) + r * 128;
+            if (r == 0) bulk_wait_read_all();  // the previous box has been read
+            named_bar_sync(bar_id, 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint4 v;
@@ -591,36 +686,32 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               v.w = __float_as_uint(__uint_as_float(o[4 * c + 3]) * inv);
               st_shared_v4(rowp + ((c ^ (r & 7)) << 4), v);
             }
+            fence_proxy_async_smem();
+            named_bar_sync(bar_id, 128);
+            if (r == 0) {
+              tma_store_3d(&tmap_o, stage, cc * 32, h * group, q0 + w.t0 + g * tpt);
+              bulk_commit_group();
+            }
           }
-          fence_proxy_async_smem();
-          named_bar_sync(bar_id, 128);
-          if (r == 0) {
+        } else {
+          float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
 #pragma unroll
-            for (int bx = 0; bx < H; ++bx)
-              tma_store_3d(&tmap_o, stage + bx * (kPfRows * 128), (rd * H + bx) * 32, h * group,
-                           q0 + t0 + g * tpt);
-            bulk_commit_group();
-            bulk_wait_read_all();
-          }
-          named_bar_sync(bar_id, 128);  // the staging buffer may be rewritten
-        }
-      } else {
-        float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+            tc_wait_ld();
+            if (valid) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
-          tc_wait_ld();
-          if (valid) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4 *>(orow + cc * 32 + e) =
-                  make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                              __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(orow + cc * 32 + e) =
+                    make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                                __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            }
           }
         }
       }
     }
+    if (r == 0) bulk_wait_read_all();  // staging is read before the CTA exits
     tc_fence_before_sync();
   }
   __syncthreads();
