@@ -99,8 +99,8 @@ bool make_q_tmap(CUtensorMap *map, const void *q, int num_tokens, int num_q_head
 }
 
 // Prefill output rows: a 3-D view [tokens][query heads][head_dim] of the
-// fp32 output, box (32 columns = 128 bytes, the GQA group's heads, tokens
-// of a tile) with the 128-byte swizzle, the layout the kernel stages O in.
+// fp32 output, box (16 columns = 64 bytes, the GQA group's heads, tokens
+// of a tile) with the 64-byte swizzle, the layout the kernel stages O in.
 bool make_out_tmap(CUtensorMap *map, float *out, int num_tokens, int num_q_heads, int head_dim,
                    int group, int tokens_per_tile) {
   auto enc = encode_fn();
@@ -109,10 +109,10 @@ bool make_out_tmap(CUtensorMap *map, float *out, int num_tokens, int num_q_heads
                         static_cast<cuuint64_t>(num_tokens)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 4,
                            static_cast<cuuint64_t>(num_q_heads) * head_dim * 4};
-  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tokens_per_tile)};
+  cuuint32_t box[3] = {16, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(tokens_per_tile)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

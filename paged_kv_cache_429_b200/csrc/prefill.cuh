@@ -106,7 +106,8 @@ struct PfPlan {
   static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int kKOff = kPfQTiles * kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr int kBoxBytes = kPfRows * 128;        // 32 fp32 columns of a tile's rows
+  static constexpr int kBoxBytes = kPfRows * 128;        // staging per query tile: 2 slots
+                                                           // of 16 fp32 columns x 128 rows
   static constexpr int kStageOff = kVOff + kVStages * kTileBytes;  // one box per query tile
   static constexpr int kBarOff = kStageOff + kPfQTiles * kBoxBytes;
   // q_full[2], q_free[2], k_full[NK], k_empty[NK], v_full[NV], v_conv[NV],
@@ -664,35 +665,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const float inv = l > 0.f ? kPfOutScale / l : 0.f;
         if (w.t0 + g * tpt + tpt <= n) {
           // Every token of the tile is in the chunk: stage O through this
-          // tile's own buffer, one box of 32 fp32 columns x the tile's rows at
-          // a time, in the 128-byte swizzled layout (thread r writes row r, its
-          // 16-byte chunk c at c ^ (r % 8): no bank conflicts), and write it
-          // with a TMA store. The last box's store drains while the next item
-          // runs; the buffer is reused only once the store has read it.
-          const uint32_t bar_id = 1 + g;
-          const uint32_t rowp = stage + r * 128;
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
-            tc_wait_ld();
-            if (r == 0) bulk_wait_read_all();  // the previous box has been read
+        // tile's own buffer, in two slots of 16 fp32 columns x the tile's
+        // rows (the 64-byte swizzled layout: thread r writes row r, its
+        // 16-byte chunk c at c ^ ((r / 2) % 4), no bank conflicts), each
+        // written by a TMA store. A slot is rewritten once the store before
+        // last has read it; the last stores drain while the next item runs.
+        const uint32_t bar_id = 1 + g;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tc_ld_32x32b_x32(trow + ocol + cc * 32, o);
+          tc_wait_ld();
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            const uint32_t slot = stage + hb * (TP::kBoxBytes / 2);
+            if (r == 0) bulk_wait_read_but_last();  // this slot's last store has read it
             named_bar_sync(bar_id, 128);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
+              const int e = 16 * hb + 4 * c;
               uint4 v;
-              v.x = __float_as_uint(__uint_as_float(o[4 * c]) * inv);
-              v.y = __float_as_uint(__uint_as_float(o[4 * c + 1]) * inv);
-              v.z = __float_as_uint(__uint_as_float(o[4 * c + 2]) * inv);
-              v.w = __float_as_uint(__uint_as_float(o[4 * c + 3]) * inv);
-              st_shared_v4(rowp + ((c ^ (r & 7)) << 4), v);
+              v.x = __float_as_uint(__uint_as_float(o[e]) * inv);
+              v.y = __float_as_uint(__uint_as_float(o[e + 1]) * inv);
+              v.z = __float_as_uint(__uint_as_float(o[e + 2]) * inv);
+              v.w = __float_as_uint(__uint_as_float(o[e + 3]) * inv);
+              st_shared_v4(slot + r * 64 + ((c ^ ((r >> 1) & 3)) << 4), v);
             }
             fence_proxy_async_smem();
             named_bar_sync(bar_id, 128);
             if (r == 0) {
-              tma_store_3d(&tmap_o, stage, cc * 32, h * group, q0 + w.t0 + g * tpt);
+              tma_store_3d(&tmap_o, slot, cc * 32 + hb * 16, h * group, q0 + w.t0 + g * tpt);
               bulk_commit_group();
             }
           }
+        }
         } else {
           float *orow = p.out + (static_cast<int64_t>(q0 + tok) * p.num_q_heads + h * group + nh) * D;
 #pragma unroll
