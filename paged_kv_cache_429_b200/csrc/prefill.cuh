@@ -127,6 +127,19 @@ __host__ __device__ constexpr uint32_t tc_idesc_f16(int M, int N, bool b_mn_majo
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// f32x2 multiply (one instruction per pair of floats).
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t y;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(a), "l"(b));
+  return y;
+}
+
+// Wait until at most the most recently committed bulk group of this thread
+// is still reading its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_but_last() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float y;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));

@@ -151,11 +151,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-// The same, but the most recently committed group may still be reading.
-__device__ __forceinline__ void bulk_wait_read_but_last() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA, tensor core) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -525,12 +520,6 @@ __device__ __forceinline__ void f2_split(uint64_t x, float &lo, float &hi) {
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t y;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y) : "l"(a), "l"(b), "l"(c));
-  return y;
-}
-
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t y;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(a), "l"(b));
   return y;
 }
 
