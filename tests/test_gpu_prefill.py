@@ -144,3 +144,17 @@ def test_prefill_mha_long_chunks_span_many_query_tiles(d):
     chunks = [1500, 300, 257, 128]
     b, q, qs = build(4, 4, d, lens, chunks, seed=5)
     check(b, q, qs, chunks)
+
+
+@pytest.mark.parametrize("scale", [6.0, 24.0])
+def test_prefill_large_scores_raise_the_running_max(scale):
+    """Queries scaled up so that scores spread over tens of units in the
+    exp2 domain: key tiles after a row's first one overflow the speculative
+    pass (their P sum passes 2^15) and are redone max first, raising the
+    running maximum and rescaling O in tensor memory, and some rows' weight
+    concentrates on a late key. The result still matches the oracle."""
+    lens = [2048, 1100, 300]
+    chunks = [2048, 600, 300]
+    b, q, qs = build(32, 8, 128, lens, chunks, seed=7)
+    q = (q.float() * scale).to(torch.bfloat16)
+    check(b, q, qs, chunks)
