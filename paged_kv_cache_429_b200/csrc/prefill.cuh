@@ -7,16 +7,20 @@
 // context_lens[s] tokens in the cache; its last n_s tokens are this chunk's
 // queries, and the query at position p attends to keys 0..p.
 //
-// Design. One CTA per (sequence, KV head, two tiles of 128 query rows); a
-// row is a (token, query head) pair with the head fastest, so the GQA
+// Design. A work item is (sequence, KV head, two tiles of 128 query rows);
+// a row is a (token, query head) pair with the head fastest, so the GQA
 // group's heads share every K/V tile and a tile fills the MMA's M = 128.
-// Both query tiles consume every K/V tile the CTA streams, so each K/V byte
-// feeds 256 rows. Keys stream in tiles of 128 (eight 16-token blocks), the
-// score MMA's N. Sixteen warps:
-//   * warp 12 (Q, K producer): 3-D TMA loads of the two tiles' Q rows, then
-//     per key tile its eight K blocks (through the block table) into a K
-//     ring freed once both tiles' scores are computed; warp 13 (V
-//     producer): the same for V into a V ring freed after both PV.
+// Both query tiles consume every K/V tile the item streams, so each K/V
+// byte feeds 256 rows. Keys stream in tiles of 128 (eight 16-token blocks),
+// the score MMA's N. A CTA takes two items of one chunk, tile pairs QT-1-x
+// and x (causal costs that sum to about the same for every CTA); its rings
+// and barrier phases run on counts over the items. Sixteen warps:
+//   * warp 12 (Q, K producer): per item 3-D TMA loads of the two tiles' Q
+//     rows (the second item's once the first item's last score MMA of that
+//     tile has completed), then per key tile its eight K blocks (through the
+//     block table) into a K ring freed once both tiles' scores are
+//     computed; warp 13 (V producer): the same for V into a V ring freed
+//     after both PV.
 //   * warps 8-11 (V widening): each landed V tile is rewritten in place as
 //     fp16 scaled by 2^-8 (exact for 2^-6 <= |v| < 2^24; smaller values keep
 //     an absolute error below 2^-17; magnitudes from 65520 * 2^8 up become
@@ -44,14 +48,15 @@
 //     with f32x2 FMAs,
 //     P is rounded to fp16 (11 significant bits) and written over the first
 //     64 score columns, and l sums P in fp32 (f32x2 adds) before rounding.
-//     At the end each thread scales its O row by 2^8 / l; a tile whose
-//     tokens all belong to the chunk is staged through its own Q buffer in
-//     the 128-byte swizzled layout and written by TMA stores (coalesced,
-//     asynchronous), other tiles row by row.
+//     At the end of an item each thread scales its O row by 2^8 / l; a tile
+//     whose tokens all belong to the chunk is staged through a private
+//     buffer of two 16-column slots in the 64-byte swizzled layout and
+//     written by TMA stores (coalesced, asynchronous, the last ones
+//     draining under the next item), other tiles row by row.
 //   * warp 15 takes part only in the register split (setmaxnreg): the two
 //     softmax warpgroups run with 192 registers, the others with 64.
-// Shared memory (head_dim 128): Q 64 KB, 2 K and 2 V stages of 32 KB:
-// 192 KB, one CTA per SM. Every wait is bounded; on time-out the kernel
+// Shared memory (head_dim 128): Q 64 KB, 2 K and 2 V stages of 32 KB, two
+// 16 KB staging buffers: 224 KB, one CTA per SM. Every wait is bounded; on time-out the kernel
 // flags PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and
 // MMAs and frees its tensor memory.
 #pragma once
