@@ -66,7 +66,7 @@
 namespace pa {
 
 constexpr int kPfRows = 128;                    // rows per query tile (MMA M)
-constexpr int kPfQTiles = 2;                    // query tiles per CTA
+constexpr int kPfQTiles = 2;                    // query tiles per work item
 constexpr int kPfKeys = 128;                    // keys per tile (S MMA N)
 constexpr int kPfBlocks = kPfKeys / kBS;        // blocks per key tile
 constexpr int kPfSoftmaxWarps = 4 * kPfQTiles;  // one warpgroup per query tile
@@ -111,9 +111,9 @@ struct PfPlan {
   static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int kKOff = kPfQTiles * kQBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr int kBoxBytes = kPfRows * 128;        // staging per query tile: 2 slots
-                                                           // of 16 fp32 columns x 128 rows
-  static constexpr int kStageOff = kVOff + kVStages * kTileBytes;  // one box per query tile
+  // output staging, per query tile: two slots of 16 fp32 columns x 128 rows
+  static constexpr int kBoxBytes = kPfRows * 128;
+  static constexpr int kStageOff = kVOff + kVStages * kTileBytes;
   static constexpr int kBarOff = kStageOff + kPfQTiles * kBoxBytes;
   // q_full[2], q_free[2], k_full[NK], k_empty[NK], v_full[NV], v_conv[NV],
   // v_empty[NV], s_full[2], p_full[2], o_done[2], drain
