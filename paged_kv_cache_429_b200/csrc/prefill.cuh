@@ -54,7 +54,8 @@
 //     written by TMA stores (coalesced, asynchronous, the last ones
 //     draining under the next item), other tiles row by row.
 //   * warp 15 takes part only in the register split (setmaxnreg): the two
-//     softmax warpgroups run with 192 registers, the others with 64.
+//     softmax warpgroups run with 184 registers, the V-widening warpgroup
+//     with 48 and the producer / MMA warpgroup with 96 (no spills).
 // Shared memory (head_dim 128): Q 64 KB, 2 K and 2 V stages of 32 KB, two
 // 16 KB staging buffers: 224 KB, one CTA per SM. Every wait is bounded; on time-out the kernel
 // flags PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and
@@ -75,9 +76,13 @@ constexpr int kPfKWarp = kPfCvtWarp0 + 4;       // Q and K loads
 constexpr int kPfVWarp = kPfKWarp + 1;          // V loads
 constexpr int kPfMmaWarp = kPfKWarp + 2;
 constexpr int kPfThreads = 16 * 32;
-constexpr int kPfSoftmaxRegs = 192;             // setmaxnreg split: 2 x 128 x 192
-constexpr int kPfOtherRegs = 64;                //   + 2 x 128 x 64 = 512 x 128
-static_assert(kPfSoftmaxRegs + kPfOtherRegs == 2 * (65536 / kPfThreads),
+// setmaxnreg split per warpgroup (128 threads each): two softmax
+// warpgroups, the V-widening warpgroup, the producer / MMA warpgroup; the
+// four shares add up to the 128 registers a thread the block launches with
+constexpr int kPfSoftmaxRegs = 184;
+constexpr int kPfCvtRegs = 48;
+constexpr int kPfMmaRegs = 96;
+static_assert(2 * kPfSoftmaxRegs + kPfCvtRegs + kPfMmaRegs == 4 * (65536 / kPfThreads),
               "register split must add up to the launch's registers");
 constexpr float kPfRescaleLog2 = 8.f;           // raise the max only past 2^8
 constexpr float kPfSpecSumMax = 32768.f;        // a speculative tile's P sums to <= 2^15
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = *s_tmem;
 
   if (warp >= kPfKWarp) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfMmaRegs));
     if (warp == kPfKWarp || warp == kPfVWarp) {
       // -------------------------------------------------------- producers
       // warp kPfKWarp: each item's Q rows (tile g's buffer reloaded once the
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
     }
   } else if (warp >= kPfCvtWarp0) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfOtherRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfCvtRegs));
     // ------------------------------------------------------- V widening
     // Thread c rewrites 16-byte chunks c, c + 128, ... of each landed V tile
     // (key row = chunk offset within its 64-dim half / 128 bytes; the
