@@ -54,8 +54,8 @@
 //     written by TMA stores (coalesced, asynchronous, the last ones
 //     draining under the next item), other tiles row by row.
 //   * warp 15 takes part only in the register split (setmaxnreg): the two
-//     softmax warpgroups run with 184 registers, the V-widening warpgroup
-//     with 48 and the producer / MMA warpgroup with 96 (no spills).
+//     softmax warpgroups run with 192 registers, the V-widening warpgroup
+//     with 40 and the producer / MMA warpgroup with 88 (no spills).
 // Shared memory (head_dim 128): Q 64 KB, 2 K and 2 V stages of 32 KB, two
 // 16 KB staging buffers: 224 KB, one CTA per SM. Every wait is bounded; on time-out the kernel
 // flags PA_DEVERR_WAIT_TIMEOUT, stops issuing, drains its own copies and
@@ -79,9 +79,9 @@ constexpr int kPfThreads = 16 * 32;
 // setmaxnreg split per warpgroup (128 threads each): two softmax
 // warpgroups, the V-widening warpgroup, the producer / MMA warpgroup; the
 // four shares add up to the 128 registers a thread the block launches with
-constexpr int kPfSoftmaxRegs = 184;
-constexpr int kPfCvtRegs = 48;
-constexpr int kPfMmaRegs = 96;
+constexpr int kPfSoftmaxRegs = 192;
+constexpr int kPfCvtRegs = 40;
+constexpr int kPfMmaRegs = 88;
 static_assert(2 * kPfSoftmaxRegs + kPfCvtRegs + kPfMmaRegs == 4 * (65536 / kPfThreads),
               "register split must add up to the launch's registers");
 constexpr float kPfRescaleLog2 = 8.f;           // raise the max only past 2^8
