@@ -48,6 +48,29 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("missing") is None
 
 
+def test_prefill_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d = tmp_path / "profiles"
+    d.mkdir()
+    f = d / "paged_prefill_16x2048.md"
+    assert bench.profiled_prefill_traffic() is None          # no profile
+    monkeypatch.setattr(bench, "prefill_source_hash", lambda: "00112233aabbccdd")
+    f.write_text("prefill_source_sha256_16: 00112233aabbccdd\ndram_bytes_per_launch: 893372416\n")
+    assert bench.profiled_prefill_traffic() == 893372416
+    monkeypatch.setattr(bench, "prefill_source_hash", lambda: "ffffffffffffffff")
+    assert bench.profiled_prefill_traffic() is None          # kernel changed since
+
+
+def test_committed_profiles_match_the_current_sources():
+    """The DRAM bytes the bench reports come from profiles taken on the
+    current kernel sources: every decode workload's and the prefill's."""
+    for w in ("llama7b", "gqa_fp8", "prefix"):
+        assert bench.profiled_traffic(w) is not None, w
+    assert bench.profiled_traffic("long", 512) is not None
+    assert bench.profiled_traffic("long", -1) is not None
+    assert bench.profiled_prefill_traffic() is not None
+
+
 def test_traffic_per_partition_size(tmp_path, monkeypatch):
     """A summary with entries per partition size gives each path its own
     bytes, and the plain entry when the size has none."""
