@@ -573,8 +573,9 @@ def test_prefill_chunks_compose():
 
 # ------------------------------------------------ block-table invariants
 #
-# The checker is the judge of the host pool, so each invariant it enforces is
-# pinned here by a hand-built table that breaks exactly that invariant. The
+# The checker decides whether the host pool is correct, so each invariant it
+# enforces is pinned here by a hand-built table that breaks exactly that
+# invariant. The
 # passing control is [Day28] §六's scenario written out by hand: request A
 # holds 20 tokens in blocks [7, 1], request B forked from it shares both
 # (refcount 2), then B's write into the partly filled block 1 copies it to
