@@ -575,11 +575,11 @@ def test_prefill_chunks_compose():
 #
 # The checker decides whether the host pool is correct, so each invariant it
 # enforces is pinned here by a hand-built table that breaks exactly that
-# invariant. The
-# passing control is [Day28] §六's scenario written out by hand: request A
-# holds 20 tokens in blocks [7, 1], request B forked from it shares both
-# (refcount 2), then B's write into the partly filled block 1 copies it to
-# block 3 (A keeps [7, 1], B gets [7, 3]; block 1's refcount drops to 1).
+# invariant. The passing control is [Day28] §六's scenario written out by
+# hand: request A holds 20 tokens in blocks [7, 1], request B forked from it
+# shares both (refcount 2), then B's write into the partly filled block 1
+# copies it to block 3 (A keeps [7, 1], B gets [7, 3]; block 1's refcount
+# drops to 1).
 
 DAY28_ROWS = [[7, 1], [7, 3]]
 DAY28_LENS = [20, 21]
