@@ -15,11 +15,15 @@ output copied back, every step; `roofline` is the decode kernel alone.
 
   python bench.py [--gpus N --steps K --warmup W --workload NAME --impl ours|reference]
                   [--fuse] [--graph] [--partition-size P] [--op step|loop|swap|prefill]
+                  [--also W[:P],... | --also none]
 
 --fuse writes the new tokens inside the decode launch (pa_decode_append);
 --graph captures one step as a CUDA graph and times its replays; --op
 selects the continuous-batching loop, block swapping or chunked prefill,
 each with its own line. --impl reference times the CPU oracle instead.
+--also measures more decode workloads in the same run (same steps and
+warm-up) and summarises each under `also`; with the default workload the
+long-context one on the automatic partitions and the fp8 one ride along.
 
 With torchrun (N > 1) every rank decodes its own batch (its own sequences,
 its own pool; no collective on the data path): weak scaling.
@@ -417,6 +421,45 @@ def run_ours(args, world, rank, local):
     return line
 
 
+def also_specs(args):
+    """The extra decode workloads of a step run: (name, partition size or
+    None for the workload's own). By default the long-context workload on
+    the automatic partitions and the fp8 one ride along with the default
+    workload, so one run measures every decode configuration's kernel."""
+    spec = args.also
+    if spec is None:
+        spec = ("long:-1,gqa_fp8" if args.workload == "llama7b" and not args.fuse
+                and not args.graph and args.partition_size is None else "none")
+    if spec.strip().lower() == "none":
+        return []
+    out = []
+    for item in spec.split(","):
+        item = item.strip()
+        if not item:
+            continue
+        name, _, ps = item.partition(":")
+        if name not in synth.WORKLOADS:
+            raise SystemExit(f"--also: unknown workload {name!r}")
+        out.append((name, int(ps) if ps else None))
+    return out
+
+
+def also_summary(line):
+    """The part of an extra workload's line kept under 'also'."""
+    r = line["roofline"]
+    return {
+        "workload": line["config"]["workload"], "dtype": line["dtype"],
+        "decode_path": line["config"]["decode_path"],
+        "partition_size": line["config"]["partition_size"],
+        "value": line["value"], "unit": line["unit"], "ms_per_step": line["ms_per_step"],
+        "tokens_per_s": line["tokens_per_s"], "e2e": line["e2e"]["value"],
+        "roofline": {k: r[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic",
+                                       "kernel", "algorithmic_bytes_per_launch",
+                                       "avg_launch_ms", "peak_source")},
+        "clocks": line["clocks"],
+    }
+
+
 def _auto_split(batch, ws) -> bool:
     """Mirror of the library's automatic choice, for reporting only."""
     w = batch.w
@@ -778,6 +821,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
                     help="capture one step in a CUDA graph and time its replays")
+    ap.add_argument("--also", default=None,
+                    help="more decode workloads measured in the same run, each WORKLOAD or "
+                         "WORKLOAD:PARTITION_SIZE, comma-separated, summarised under 'also' "
+                         "(default with the default workload: long:-1,gqa_fp8; 'none' for none)")
     ap.add_argument("--fuse", action="store_true",
                     help="write the new tokens inside the decode launch (pa_decode_append) "
                          "instead of a separate pa_reshape_and_cache launch")
@@ -802,7 +849,21 @@ def main(argv=None):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     try:
         line = run_ours(args, world, rank, local)
+        also = []
+        for wname, ps in also_specs(args):
+            import copy
+            import gc
+            gc.collect()
+            torch.cuda.empty_cache()
+            sub_args = copy.copy(args)
+            sub_args.workload, sub_args.partition_size = wname, ps
+            sub_args.no_cpu_baseline, sub_args.fuse, sub_args.graph = True, False, False
+            sub = run_ours(sub_args, world, rank, local)
+            if sub is not None:
+                also.append(also_summary(sub))
         if line is not None:
+            if also:
+                line["also"] = also
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

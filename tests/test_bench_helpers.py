@@ -124,3 +124,19 @@ def test_reference_arm_other_ranks_print_nothing(capsys, monkeypatch):
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--steps", "3", "--warmup", "2"])
+
+
+def test_also_specs():
+    import argparse
+    ns = argparse.Namespace(also=None, workload="llama7b", fuse=False, graph=False,
+                            partition_size=None)
+    assert bench.also_specs(ns) == [("long", -1), ("gqa_fp8", None)]
+    ns.fuse = True                      # a non-default run adds nothing by itself
+    assert bench.also_specs(ns) == []
+    ns.also = "prefix, long:512"
+    assert bench.also_specs(ns) == [("prefix", None), ("long", 512)]
+    ns.also = "none"
+    assert bench.also_specs(ns) == []
+    ns.also = "nosuch"
+    with pytest.raises(SystemExit):
+        bench.also_specs(ns)
